@@ -1,0 +1,178 @@
+// The C ABI (include/attn.h): argument checks, TMA descriptors, launches, the device error word.
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <mutex>
+
+#include "attn_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace attn {
+
+__device__ unsigned int g_error_word = 0;
+
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                            uint64_t limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 256; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (abort_flag != nullptr && *abort_flag) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      atomicOr(&g_error_word, kErrTimeoutBit);
+      if (abort_flag != nullptr) *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+// One CTA waits on a barrier that is initialised for one arrival and never receives it.
+__global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, limit_ns);
+  __syncthreads();
+}
+
+// ---- driver entry point for cuTensorMapEncodeTiled (no link-time dependency on libcuda) ----
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool encode_tile_map(CUtensorMap* map, const void* base, int d, int heads, int rows, int outer, int box_cols,
+                     int box_rows, unsigned swizzle_bytes) {
+  auto fn = get_encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(heads), cuuint64_t(rows), cuuint64_t(outer)};
+  const cuuint64_t strides[3] = {cuuint64_t(d) * 2, cuuint64_t(heads) * d * 2, cuuint64_t(rows) * heads * d * 2};
+  const cuuint32_t box[4] = {cuuint32_t(box_cols), 1u, cuuint32_t(box_rows), 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" {
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                       int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
+  if (d != 32 && d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  return fwd_dispatch(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, stream);
+}
+
+int attn_decode_default_chunk(int B, int Hkv, int Nkv_cap) {
+  if (B < 1 || Hkv < 1 || Nkv_cap < 1) return 0;
+  return decode_default_chunk(B, Hkv, Nkv_cap);
+}
+
+size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int Nkv_cap, int chunk) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || d < 1 || Nkv_cap < 1 || chunk < 0 || Hq % Hkv) return 0;
+  if (chunk == 0) chunk = decode_default_chunk(B, Hkv, Nkv_cap);
+  return decode_workspace(B, Hq, d, Nkv_cap, chunk);
+}
+
+attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, const int32_t* kv_lens,
+                                  int Nkv_cap, void* o, float* lse, int B, int Hq, int Hkv, int d, float scale,
+                                  int chunk, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!q || !k_cache || !v_cache || !kv_lens || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(kv_lens) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nkv_cap < 1 || Hq % Hkv != 0 || chunk < 0 || (chunk % 64) != 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  const int G = Hq / Hkv;
+  if ((d != 64 && d != 128 && d != 256) || (G != 1 && G != 2 && G != 4 && G != 8)) return ATTN_ERR_UNSUPPORTED;
+  if (chunk == 0) chunk = decode_default_chunk(B, Hkv, Nkv_cap);
+  const long long n_splits = (Nkv_cap + (long long)chunk - 1) / chunk;
+  const size_t need = decode_workspace(B, Hq, d, Nkv_cap, chunk);
+  if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  if (Hkv > 65535 || B > 65535) return ATTN_ERR_UNSUPPORTED;
+  float* po = static_cast<float*>(workspace);
+  const size_t po_bytes = size_t(B) * Hq * n_splits * d * sizeof(float);
+  float* pl = reinterpret_cast<float*>(static_cast<char*>(workspace) + ((po_bytes + 255) / 256) * 256);
+  attn_status_t st =
+      decode_split_dispatch(q, k_cache, v_cache, kv_lens, Nkv_cap, B, Hq, Hkv, d, scale, chunk, int(n_splits), po,
+                            pl, stream);
+  if (st != ATTN_OK) return st;
+  return decode_combine_dispatch(po, pl, B * Hq, int(n_splits), d, o, lse, stream);
+}
+
+attn_status_t attn_decode_combine(const float* part_o, const float* part_lse, int rows, int n_splits, int d,
+                                  void* o, float* lse, cudaStream_t stream) {
+  if (!part_o || !part_lse || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(part_o) || !aligned16(o) || (reinterpret_cast<uintptr_t>(part_lse) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (rows < 1 || n_splits < 1) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  return decode_combine_dispatch(part_o, part_lse, rows, n_splits, d, o, lse, stream);
+}
+
+attn_status_t attn_get_last_error(void) {
+  unsigned int word = 0;
+  const unsigned int zero = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (word & kErrTimeoutBit) return ATTN_ERR_TIMEOUT;
+  if (word & kErrBadLengthBit) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+const char* attn_status_string(attn_status_t s) {
+  switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ATTN_ERR_WORKSPACE: return "decode workspace missing or too small";
+    case ATTN_ERR_CUDA: return "CUDA call failed";
+    case ATTN_ERR_TIMEOUT: return "a kernel pipeline wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* attn_kernel_name(int which) {
+  switch (which) {
+    case 0: return "attn::attn_fwd_kernel<D>";
+    case 1: return "attn::decode_split_kernel<D,G>";
+    case 2: return "attn::decode_combine_kernel<D>";
+  }
+  return nullptr;
+}
+
+attn_status_t attn_selftest_bounded_wait(unsigned int limit_us, cudaStream_t stream) {
+  if (limit_us == 0 || limit_us > 10000000u) return ATTN_ERR_INVALID_ARG;
+  bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(1000ull * limit_us);
+  return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
+}
+
+}  // extern "C"

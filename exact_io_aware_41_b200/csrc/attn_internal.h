@@ -1,0 +1,49 @@
+// Declarations shared by the library's translation units (not part of the public ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/attn.h"
+
+namespace attn {
+
+// Bits of the device error word (g_error_word).
+enum : unsigned int {
+  kErrBadLengthBit = 2u,  // a decode length outside [0, Nkv_cap] was clamped
+};
+
+// Wall-time limit of every pipeline wait inside a kernel. Far above any legitimate wait (a whole
+// 8k x 8k head takes well under a millisecond), so reaching it means the pipeline is broken.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+struct FwdArgs {
+  void* o;
+  float* lse;
+  int B, Hq, Hkv, Nq, Nkv;
+  int group;   // Hq / Hkv
+  int n_qblk;  // query blocks of NQT*128 rows per (b, h)
+  int causal;
+  float scale;       // natural-log scale on Q K^T
+  float scale_log2;  // scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+// A 4-d TMA map over a token-major bf16 tensor [outer, rows, heads, d] (d innermost), with a box
+// of `box_cols` elements of d x 1 head x `box_rows` tokens x 1 batch. Returns false on failure.
+bool encode_tile_map(CUtensorMap* map, const void* base, int d, int heads, int rows, int outer, int box_cols,
+                     int box_rows, unsigned swizzle_bytes);
+
+attn_status_t fwd_dispatch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                           int Hkv, int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream);
+
+int decode_default_chunk(int B, int Hkv, int Nkv_cap);
+size_t decode_workspace(int B, int Hq, int d, int Nkv_cap, int chunk);
+attn_status_t decode_split_dispatch(const void* q, const void* kc, const void* vc, const int32_t* lens, int cap,
+                                    int B, int Hq, int Hkv, int d, float scale, int chunk, int n_splits,
+                                    float* po, float* pl, cudaStream_t st);
+attn_status_t decode_combine_dispatch(const float* po, const float* pl, int rows, int n_splits, int d, void* o,
+                                      float* lse, cudaStream_t st);
+
+}  // namespace attn

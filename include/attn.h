@@ -1,0 +1,139 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) exact-attention library.
+ *
+ * The library computes exact scaled-dot-product attention,
+ *     O = softmax(scale * Q K^T) V,   LSE[i] = log sum_j exp(scale * q_i . k_j),
+ * tile by tile with the online-softmax recurrence, so the N x N score and probability matrices
+ * never reach HBM (the invariant of every FlashAttention version: "FlashAttention evolution"
+ * article, section 1 "The Invariant and the Moving Bottleneck"; the per-row metadata beside O:
+ * "Flash Attention" overview, section "The IO problem").
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ *  - All tensors live in device memory owned by the caller. The library allocates nothing per call
+ *    and keeps no pointer after a call returns. Work is enqueued on `stream` and runs
+ *    asynchronously; no entry point synchronises the host.
+ *  - bf16 tensors are dense and token-major:
+ *        Q, O   [B, Nq, Hq, d]        K, V   [B, Nkv, Hkv, d]         LSE [B, Hq, Nq] (fp32)
+ *    Decode: q, O [B, Hq, d]; caches [B, Nkv_cap, Hkv, d]; kv_lens int32 [B]; LSE [B, Hq].
+ *  - Every pointer must be 16-byte aligned. d must be 32, 64, 128 or 256. Hq must be a multiple of
+ *    Hkv; query head h reads kv head h / (Hq / Hkv) (contiguous groups).
+ *  - Causal masking is bottom-right aligned: key j is visible to query i iff j <= i + Nkv - Nq.
+ *    A query row that sees no key gets O = 0 and LSE = -inf.
+ *  - Arithmetic: bf16 inputs, fp32 accumulation and softmax state, bf16 O, fp32 LSE in natural log.
+ *  - Errors: argument errors are reported before anything is enqueued. Launch failures map to
+ *    ATTN_ERR_CUDA. Kernel-side faults that the kernels detect themselves (a pipeline wait that
+ *    gave up, an out-of-range decode length) are recorded in a device error word read by
+ *    attn_get_last_error(). No entry point throws, aborts or traps.
+ */
+#ifndef EXACT_IO_AWARE_ATTN_H
+#define EXACT_IO_AWARE_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, non-positive size, Hq % Hkv != 0, ... */
+  ATTN_ERR_UNSUPPORTED = 2, /* a head dim or GQA group the kernels are not built for */
+  ATTN_ERR_WORKSPACE = 3,   /* decode workspace missing or smaller than attn_decode_workspace_bytes */
+  ATTN_ERR_CUDA = 4,        /* a CUDA runtime or driver call failed (launch, attribute, tensor map) */
+  ATTN_ERR_TIMEOUT = 5      /* a kernel's bounded pipeline wait gave up (reported by attn_get_last_error) */
+} attn_status_t;
+
+/*
+ * Prefill forward: O = softmax(scale * Q K^T) V and LSE, causal or not, with GQA.
+ * ("FlashAttention evolution", sections 3-5: query-block parallelism, producer/consumer overlap,
+ *  accumulators in tensor memory.)
+ *
+ *   q      [B, Nq, Hq, d]  bf16, read only
+ *   k, v   [B, Nkv, Hkv, d] bf16, read only
+ *   o      [B, Nq, Hq, d]  bf16, written
+ *   lse    [B, Hq, Nq]     fp32, written (natural-log log-sum-exp of the scaled scores)
+ *   B, Hq, Hkv, Nq, Nkv >= 1; d in {32, 64, 128, 256}; scale > 0 and finite (1/sqrt(d) usually);
+ *   causal 0 or 1.
+ * Returns ATTN_OK once the kernel is enqueued.
+ */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                       int Hkv, int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream);
+
+/*
+ * Bytes of device workspace attn_decode_splitkv needs: the per-split partial outputs
+ * (fp32 [B, Hq, n_splits, d]) and partial LSEs (fp32 [B, Hq, n_splits]), n_splits =
+ * ceil(Nkv_cap / chunk). chunk = 0 selects the same automatic chunk attn_decode_splitkv uses.
+ * Returns 0 for invalid arguments.
+ */
+size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int d, int Nkv_cap, int chunk);
+
+/* The KV chunk (tokens per split) chosen when chunk = 0 is passed. */
+int attn_decode_default_chunk(int B, int Hkv, int Nkv_cap);
+
+/*
+ * Flash-Decoding split-KV forward for one query token per sequence, followed by the LSE-weighted
+ * combine, both enqueued on `stream` ("FlashAttention evolution", section 6 "Flash-Decoding: A
+ * Different Parallel Shape": partitions of the KV sequence each produce a partial max, sum and
+ * weighted output; a final reduction merges them with the online-softmax identity).
+ *
+ *   q                [B, Hq, d] bf16
+ *   k_cache, v_cache [B, Nkv_cap, Hkv, d] bf16; only tokens [0, kv_lens[b]) of sequence b are read
+ *   kv_lens          int32 [B] in device memory, each in [0, Nkv_cap] (out-of-range values are
+ *                    clamped and flagged in the device error word)
+ *   o                [B, Hq, d] bf16, written;  lse [B, Hq] fp32, written (-inf when kv_lens[b] = 0)
+ *   d in {64, 128, 256}; Hq / Hkv in {1, 2, 4, 8}; chunk = tokens per split (multiple of 64) or 0.
+ *   workspace        caller-owned device memory of at least attn_decode_workspace_bytes(...) bytes;
+ *                    fully overwritten before it is read, so it needs no initialisation.
+ */
+attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* kv_lens, int Nkv_cap, void* o, float* lse, int B, int Hq,
+                                  int Hkv, int d, float scale, int chunk, void* workspace,
+                                  size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * The combine step on its own: merges n_splits partial states per row with
+ *     LSE = log sum_s exp(lse_s),   O = sum_s exp(lse_s - LSE) * o_s
+ * ("FlashAttention evolution", section 6). Partials with lse_s = -inf contribute nothing; a row
+ * whose partials are all -inf gets O = 0 and LSE = -inf.
+ *
+ *   part_o   fp32 [rows, n_splits, d] (each o_s already normalised by its own sum)
+ *   part_lse fp32 [rows, n_splits]
+ *   o        bf16 [rows, d], written;  lse fp32 [rows], written
+ *   rows >= 1, n_splits >= 1, d in {64, 128, 256}.
+ */
+attn_status_t attn_decode_combine(const float* part_o, const float* part_lse, int rows, int n_splits, int d,
+                                  void* o, float* lse, cudaStream_t stream);
+
+/*
+ * Reads and clears the device error word (synchronises the calling thread with the device).
+ * ATTN_OK if no kernel recorded a fault since the last call, ATTN_ERR_TIMEOUT if a bounded
+ * pipeline wait gave up, ATTN_ERR_INVALID_ARG if a decode length was out of range, ATTN_ERR_CUDA
+ * if the word could not be read.
+ */
+attn_status_t attn_get_last_error(void);
+
+/* Static, human-readable name of a status code. */
+const char* attn_status_string(attn_status_t status);
+
+/*
+ * Name of the kernel that `which` selects (0 = prefill forward, 1 = decode split, 2 = decode
+ * combine), for recording which kernel a measurement ran (the evolution article's section 1.1
+ * asks that a benchmark name its kernel). Returns NULL for an unknown index.
+ */
+const char* attn_kernel_name(int which);
+
+/*
+ * Test hook for the bounded waits: launches a one-CTA kernel that waits on an mbarrier nothing
+ * ever completes, with the given limit in microseconds, then returns normally. Afterwards
+ * attn_get_last_error() reports ATTN_ERR_TIMEOUT. Nothing faults or hangs.
+ */
+attn_status_t attn_selftest_bounded_wait(unsigned int limit_us, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_IO_AWARE_ATTN_H */

@@ -1,0 +1,103 @@
+"""The C-ABI library builds, loads, and exports every entry point include/attn.h declares.
+
+No call here reaches the GPU: only pure host functions and argument checks that fail before any
+CUDA call are exercised.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    with open(os.path.join(ROOT, "include", "attn.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def raw():
+    from exact_io_aware_41_b200 import build
+
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for must in ("attn_fwd", "attn_decode_splitkv", "attn_decode_combine", "attn_decode_workspace_bytes",
+                 "attn_get_last_error", "attn_status_string", "attn_kernel_name"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(raw):
+    for name in _declared_functions():
+        assert hasattr(raw, name), name
+
+
+def test_binding_covers_every_declared_symbol(raw):
+    import exact_io_aware_41_b200 as pkg
+
+    assert set(_declared_functions()) == set(pkg.SIGNATURES)
+    for name in _declared_functions():
+        assert callable(getattr(pkg, name, None)) or name in ("attn_status_string", "attn_kernel_name")
+
+
+def test_status_strings_and_kernel_names():
+    import exact_io_aware_41_b200 as pkg
+
+    assert pkg.status_string(0) == "ok"
+    assert "timed out" in pkg.status_string(pkg.ATTN_ERR_TIMEOUT)
+    assert pkg.status_string(99) == "unknown status"
+    assert pkg.kernel_name(0).startswith("attn::attn_fwd_kernel")
+    assert pkg.kernel_name(1).startswith("attn::decode_split_kernel")
+    assert pkg.kernel_name(7) is None
+
+
+def test_decode_workspace_sizing():
+    import exact_io_aware_41_b200 as pkg
+
+    # n_splits = ceil(1000 / 64) = 16; part_o = 2*8*16*128*4 = 131072 bytes (already 256-aligned);
+    # part_lse = 2*8*16*4 = 1024 bytes
+    assert pkg.attn_decode_workspace_bytes(2, 8, 2, 128, 1000, 64) == 131072 + 1024
+    assert pkg.attn_decode_workspace_bytes(0, 8, 2, 128, 1000, 64) == 0
+    assert pkg.attn_decode_workspace_bytes(2, 8, 3, 128, 1000, 64) == 0
+    c = pkg.attn_decode_default_chunk(8, 8, 131072)
+    assert c % 64 == 0 and 64 <= c <= 512
+    assert pkg.attn_decode_workspace_bytes(8, 32, 8, 128, 131072, 0) == \
+        pkg.attn_decode_workspace_bytes(8, 32, 8, 128, 131072, c)
+
+
+def test_argument_errors_are_reported_before_any_launch(raw):
+    import exact_io_aware_41_b200 as pkg
+
+    lib = pkg._lib
+    p = 1 << 20  # aligned, never dereferenced: every call below fails validation first
+    # null pointer
+    assert lib.attn_fwd(0, p, p, p, p, 1, 2, 2, 16, 16, 64, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG
+    # misaligned pointer
+    assert lib.attn_fwd(p + 2, p, p, p, p, 1, 2, 2, 16, 16, 64, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG
+    # Hq not a multiple of Hkv, zero sizes, bad scale, bad causal flag
+    assert lib.attn_fwd(p, p, p, p, p, 1, 3, 2, 16, 16, 64, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd(p, p, p, p, p, 1, 2, 2, 0, 16, 64, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd(p, p, p, p, p, 1, 2, 2, 16, 16, 64, -1.0, 0, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd(p, p, p, p, p, 1, 2, 2, 16, 16, 64, float("nan"), 0, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd(p, p, p, p, p, 1, 2, 2, 16, 16, 64, 0.125, 2, None) == pkg.ATTN_ERR_INVALID_ARG
+    # unsupported head dim
+    assert lib.attn_fwd(p, p, p, p, p, 1, 2, 2, 16, 16, 48, 0.125, 0, None) == pkg.ATTN_ERR_UNSUPPORTED
+    # decode: chunk not a multiple of 64, unsupported group, too little workspace
+    args = [p, p, p, p, 1024, p, p, 2, 8, 2, 128, 0.1]
+    assert lib.attn_decode_splitkv(*args, 100, p, 1 << 30, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert lib.attn_decode_splitkv(p, p, p, p, 1024, p, p, 2, 6, 2, 128, 0.1, 64, p, 1 << 30, None) == \
+        pkg.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_decode_splitkv(p, p, p, p, 1024, p, p, 2, 8, 2, 32, 0.1, 64, p, 1 << 30, None) == \
+        pkg.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_decode_splitkv(*args, 64, p, 16, None) == pkg.ATTN_ERR_WORKSPACE
+    assert lib.attn_decode_splitkv(*args, 64, 0, 1 << 30, None) == pkg.ATTN_ERR_WORKSPACE
+    assert lib.attn_decode_combine(p, p, 0, 4, 128, p, p, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert lib.attn_decode_combine(p, p, 4, 4, 96, p, p, None) == pkg.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_selftest_bounded_wait(0, None) == pkg.ATTN_ERR_INVALID_ARG

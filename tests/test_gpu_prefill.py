@@ -1,0 +1,115 @@
+"""Prefill parity: the CUDA path (through the C ABI) against the fp64 CPU oracle on the same seeded
+bf16 inputs. Small shapes are compared element by element over the whole output; the full-size
+workloads are compared on sampled rows the oracle computes one by one, plus properties that hold
+at any size."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from parity import (assert_parity, bf16_tensor_to_f64, draw_prefill, kv_slice_bits, oracle_rows_prefill,
+                    sample_rows, to_torch_bf16)
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_small(lib, seed, B, Hq, Hkv, Nq, Nkv, d, causal, scale=None):
+    import torch
+
+    qb, kb, vb = draw_prefill(seed, B, Hq, Hkv, Nq, Nkv, d)
+    sc = scale if scale is not None else 1.0 / math.sqrt(d)
+    o, lse = lib.attn_fwd(to_torch_bf16(qb), to_torch_bf16(kb), to_torch_bf16(vb), scale=sc, causal=causal)
+    torch.cuda.synchronize()
+    O_ref, L_ref = oracle.attention(synth.bf16_bits_to_f64(qb), synth.bf16_bits_to_f64(kb),
+                                    synth.bf16_bits_to_f64(vb), sc, causal)
+    what = f"B{B} Hq{Hq} Hkv{Hkv} Nq{Nq} Nkv{Nkv} d{d} causal={causal}"
+    lse_g = lse.cpu().numpy().astype(np.float64).transpose(0, 2, 1)
+    assert_parity(bf16_tensor_to_f64(o), lse_g, O_ref, L_ref.transpose(0, 2, 1), what)
+    assert lib.attn_get_last_error() == lib.ATTN_OK
+
+
+def test_tiny_workload(lib):
+    w = synth.TINY
+    _run_small(lib, w.seed, w.B, w.Hq, w.Hkv, w.Nq, w.Nkv, w.d, w.causal)
+
+
+@pytest.mark.parametrize("d", [32, 64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_every_head_dim_ragged_tiles(lib, d, causal):
+    # 300 rows/keys: several 128-row tiles and a ragged tail; GQA group of 2
+    _run_small(lib, 2000 + d, 2, 4, 2, 300, 300, d, causal)
+
+
+@pytest.mark.parametrize("Nq,Nkv,causal", [
+    (1, 777, False), (1, 777, True), (130, 513, True), (600, 200, True), (5, 5, False), (5, 5, True),
+    (256, 1, False), (257, 129, False), (64, 1000, True),
+])
+def test_edge_shapes(lib, Nq, Nkv, causal):
+    _run_small(lib, 3000 + Nq + Nkv, 1, 2, 1, Nq, Nkv, 128, causal)
+
+
+@pytest.mark.parametrize("d", [64, 256])
+def test_edge_shapes_other_head_dims(lib, d):
+    _run_small(lib, 3100 + d, 1, 2, 2, 1, 300, d, True)
+    _run_small(lib, 3200 + d, 1, 2, 2, 200, 70, d, True)
+
+
+def test_gqa_group_of_eight_causal(lib):
+    _run_small(lib, 4000, 1, 8, 1, 384, 384, 128, True)
+
+
+def test_large_score_spread(lib):
+    # scale far above 1/sqrt(d) makes the running max jump often, exercising the O rescale path
+    _run_small(lib, 4100, 1, 2, 2, 512, 512, 128, False, scale=1.5)
+    _run_small(lib, 4101, 1, 2, 2, 512, 512, 128, True, scale=1.5)
+    _run_small(lib, 4102, 1, 2, 2, 384, 384, 256, True, scale=1.5)
+
+
+def test_repeat_calls_are_identical(lib):
+    import torch
+
+    qb, kb, vb = draw_prefill(4200, 1, 4, 4, 512, 512, 128)
+    q, k, v = to_torch_bf16(qb), to_torch_bf16(kb), to_torch_bf16(vb)
+    o1, l1 = lib.attn_fwd(q, k, v, causal=True)
+    o1, l1 = o1.clone(), l1.clone()
+    for _ in range(5):
+        o2, l2 = lib.attn_fwd(q, k, v, causal=True)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+FULL = [synth.CAUSAL_2K, synth.LONG_8K, synth.LONG_8K_CAUSAL, synth.LONG_8K_GQA, synth.LONG_8K_GQA_CAUSAL,
+        *synth.SWEEP]
+
+
+@pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
+def test_full_size_workload_sampled_rows(lib, w):
+    import torch
+
+    dev = "cuda"
+    q = synth.normal_bf16_torch(w.seed, synth.STREAM_Q, (w.B, w.Nq, w.Hq, w.d), dev)
+    k = synth.normal_bf16_torch(w.seed, synth.STREAM_K, (w.B, w.Nkv, w.Hkv, w.d), dev)
+    v = synth.normal_bf16_torch(w.seed, synth.STREAM_V, (w.B, w.Nkv, w.Hkv, w.d), dev)
+    # the device draw is the host draw (checked on one kv row block)
+    host = kv_slice_bits(w.seed, synth.STREAM_K, tuple(k.shape), w.B - 1, w.Hkv - 1, 256)
+    assert np.array_equal(k[w.B - 1, :256, w.Hkv - 1].cpu().view(torch.int16).numpy().view(np.uint16), host)
+
+    o, lse = lib.attn_fwd(q, k, v, scale=w.scale, causal=w.causal)
+    torch.cuda.synchronize()
+    assert lib.attn_get_last_error() == lib.ATTN_OK
+
+    # properties at full size: finite, and each O element inside the range of V over its kv head
+    assert torch.isfinite(o.float()).all()
+    assert torch.isfinite(lse).all()
+    vmax = v.float().abs().amax().item()
+    assert o.float().abs().amax().item() <= vmax * (1 + 2 ** -6)
+
+    rng = np.random.default_rng(w.seed)
+    picks = sample_rows(rng, w.B, w.Nq, w.Hq, 48, w.causal)
+    O_ref, L_ref = oracle_rows_prefill(w, picks)
+    idx = tuple(np.array(p) for p in zip(*picks))
+    o_s = bf16_tensor_to_f64(o[idx[0], idx[1], idx[2]])
+    l_s = lse[idx[0], idx[2], idx[1]].cpu().numpy().astype(np.float64)
+    assert_parity(o_s, l_s, O_ref, L_ref, w.name)
