@@ -1,0 +1,628 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200; prints one JSON line on rank 0.
+
+A step is one pass over both entry points of the hot path:
+  * prefill: attn_fwd on the causal workload B=4, H=16, N=2048, d=128 (bf16, scale 1/sqrt(d));
+  * decode:  attn_decode_splitkv (split kernel + combine) on B=8, Hq=32, Hkv=8, d=128 with KV
+             lengths drawn uniformly from [1024, 131072].
+`value` is the prefill throughput in TFLOP/s (causal FLOPs = half of 4*B*H*N^2*d); the decode half
+of the metric is reported under "decode" in GB/s of algorithmic HBM bytes. Both are timed with CUDA
+events on the launching stream; the step's inputs (2.3 GB) exceed the 126 MB L2, and the decode pass
+evicts the prefill inputs before the next step. "gates" times the long-sequence prefill workloads
+(N=8192) and the head-dim sweep the same way.
+
+`--impl reference` times the CPU oracle instead, on a bounded sample of the same workloads.
+Multi-GPU (torchrun): every rank runs the same step on its own GPU (independent problems, no
+collective on the data path); `value` counts the work of all ranks over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "attn fwd TFLOP/s & % of BF16 peak (prefill); decode HBM GB/s & % of peak"
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], 0.0, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = max(smax, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------------
+# distributed plumbing
+# ------------------------------------------------------------------------------------------------
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=None)
+        pg = dist
+    return world, rank, local, pg
+
+
+def physical_gpu(local: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x for x in vis.split(",") if x.strip()]
+        if local < len(ids) and ids[local].strip().isdigit():
+            return int(ids[local])
+    return local
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ------------------------------------------------------------------------------------------------
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def _head_inputs(w: synth.Prefill, b: int, h: int):
+    g = h // (w.Hq // w.Hkv)
+    dq = np.arange(w.d, dtype=np.int64)
+    tq = np.arange(w.Nq, dtype=np.int64)[:, None]
+    tk = np.arange(w.Nkv, dtype=np.int64)[:, None]
+    q = synth.normal_bf16_at(w.seed, synth.STREAM_Q, (((b * w.Nq + tq) * w.Hq + h) * w.d + dq).reshape(-1))
+    kidx = (((b * w.Nkv + tk) * w.Hkv + g) * w.d + dq).reshape(-1)
+    k = synth.normal_bf16_at(w.seed, synth.STREAM_K, kidx)
+    v = synth.normal_bf16_at(w.seed, synth.STREAM_V, kidx)
+    f = synth.bf16_bits_to_f64
+    return (f(q).reshape(1, w.Nq, 1, w.d), f(k).reshape(1, w.Nkv, 1, w.d), f(v).reshape(1, w.Nkv, 1, w.d))
+
+
+def cpu_prefill(w: synth.Prefill, budget_s: float):
+    import oracle
+
+    heads, flops, spent = 0, 0.0, 0.0
+    per_head = w.flops / (w.B * w.Hq)
+    while spent < budget_s and heads < w.B * w.Hq:
+        b, h = divmod(heads, w.Hq)
+        q, k, v = _head_inputs(w, b, h)
+        t0 = time.perf_counter()
+        oracle.attention(q, k, v, w.scale, w.causal)
+        spent += time.perf_counter() - t0
+        flops += per_head
+        heads += 1
+    return flops / spent / 1e12, f"{heads} of {w.B * w.Hq} (b, h) heads of {w.name}, {spent:.1f} s", spent
+
+
+def cpu_decode(w: synth.Decode, budget_s: float, tokens: int = 16384):
+    """Oracle decode on batch row 0 truncated to `tokens` KV tokens, repeated until the budget is spent."""
+    import oracle
+
+    L = min(tokens, int(w.lengths()[0]))
+    cap = L
+    shape = (1, cap, w.Hkv, w.d)
+    q = synth.bf16_bits_to_f64(synth.normal_bf16(w.seed, synth.STREAM_Q, (1, w.Hq, w.d)))
+    k = synth.bf16_bits_to_f64(synth.normal_bf16(w.seed, synth.STREAM_K, shape))
+    v = synth.bf16_bits_to_f64(synth.normal_bf16(w.seed, synth.STREAM_V, shape))
+    byts, spent, reps = 0.0, 0.0, 0
+    while spent < budget_s:
+        t0 = time.perf_counter()
+        oracle.decode(q, k, v, np.array([L]), w.scale)
+        spent += time.perf_counter() - t0
+        byts += L * w.Hkv * w.d * 2 * 2
+        reps += 1
+    return byts / spent / 1e9, f"{reps} x (batch row 0, first {L} KV tokens, all {w.Hq} heads) of {w.name}", spent
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------------
+def run_ours(args, world, rank, local, dist):
+    import torch
+
+    import exact_io_aware_41_b200 as lib
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    peaks, peak_src = _peaks()
+
+    P = synth.CAUSAL_2K
+    Dw = synth.DECODE
+    q = synth.normal_bf16_torch(P.seed, synth.STREAM_Q, (P.B, P.Nq, P.Hq, P.d), dev)
+    k = synth.normal_bf16_torch(P.seed, synth.STREAM_K, (P.B, P.Nkv, P.Hkv, P.d), dev)
+    v = synth.normal_bf16_torch(P.seed, synth.STREAM_V, (P.B, P.Nkv, P.Hkv, P.d), dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((P.B, P.Hq, P.Nq), dtype=torch.float32, device=dev)
+
+    cap = Dw.cap
+    lens_np = Dw.lengths()
+    dq = synth.normal_bf16_torch(Dw.seed, synth.STREAM_Q, (Dw.B, Dw.Hq, Dw.d), dev)
+    kc = synth.normal_bf16_torch(Dw.seed, synth.STREAM_K, (Dw.B, cap, Dw.Hkv, Dw.d), dev)
+    vc = synth.normal_bf16_torch(Dw.seed, synth.STREAM_V, (Dw.B, cap, Dw.Hkv, Dw.d), dev)
+    lens = torch.from_numpy(lens_np).to(dev)
+    do = torch.empty_like(dq)
+    dlse = torch.empty((Dw.B, Dw.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(lib.attn_decode_workspace_bytes(Dw.B, Dw.Hq, Dw.Hkv, Dw.d, cap, 0), dtype=torch.uint8,
+                     device=dev)
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    K, W = args.steps, args.warmup
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+
+    def step(e=None):
+        if e is not None:
+            e[0].record(stream)
+        lib.attn_fwd(q, k, v, scale=P.scale, causal=P.causal, out=o, lse=lse)
+        if e is not None:
+            e[1].record(stream)
+        lib.attn_decode_splitkv(dq, kc, vc, lens, scale=Dw.scale, workspace=ws, out=do, lse=dlse)
+        if e is not None:
+            e[2].record(stream)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    sampler = ClockSampler(physical_gpu(local))
+    sampler.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    for i in range(K):
+        step(ev[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    pf_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+    dec_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
+    times = torch.tensor([total_ms, pf_ms, dec_ms], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    total_ms, pf_ms, dec_ms = times.tolist()
+    err = lib.attn_get_last_error()
+    if err != lib.ATTN_OK:
+        raise SystemExit(f"device error word after the timed region: {lib.status_string(err)}")
+
+    pf_flops = P.flops
+    dec_bytes = Dw.algorithmic_bytes()
+    value = world * K * pf_flops / (pf_ms * 1e-3) / 1e12
+    pf_avg_s = pf_ms * 1e-3 / K
+    dec_avg_s = dec_ms * 1e-3 / K
+    pf_tflops_1 = pf_flops / pf_avg_s / 1e12
+    dec_gbs_1 = dec_bytes / dec_avg_s / 1e9
+    dec_value = world * K * dec_bytes / (dec_ms * 1e-3) / 1e9
+
+    # ---- gates: long-sequence prefill and head-dim sweep (same timing, not part of `value`)
+    gates = {}
+    if not args.no_gates:
+        for w in (synth.LONG_8K, synth.LONG_8K_CAUSAL, synth.LONG_8K_GQA, synth.LONG_8K_GQA_CAUSAL,
+                  *synth.SWEEP):
+            gates[w.name] = time_prefill(lib, w, dev, stream, peaks)
+            torch.cuda.empty_cache()
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e = e2e_prefill(lib, P, q, k, v, stream, max(3, min(K, 50)))
+    dec_e2e = e2e_decode(lib, Dw, dq, kc, vc, lens_np, stream, 2) if not args.no_e2e_decode else None
+    if dist:
+        t = torch.tensor([e2e["ms"], (dec_e2e or {}).get("ms", 0.0)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e["ms"], dms = t.tolist()
+        if dec_e2e:
+            dec_e2e["ms"] = dms
+
+    if rank != 0:
+        return None
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        v_cpu, sample, _ = cpu_prefill(P, args.cpu_budget)
+        cpu = {"value": v_cpu, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle", "sample": sample}
+        dv, dsample, _ = cpu_decode(Dw, args.cpu_budget / 2)
+        cpu["decode"] = {"value": dv, "unit": "GB/s", "sample": dsample}
+
+    meas_tf = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
+    meas_bw = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": total_ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic: seeded i.i.d. N(0,1) rounded to bf16 (splitmix64 + Box-Muller), decode lengths U[1024,131072]",
+        "config": {
+            "workload": P.name,
+            "decode_workload": Dw.name,
+            "decode_kv_tokens": int(lens_np.sum()),
+            "parallelism": f"replica x{world} (independent problems, no collective)",
+            "l2": "inputs larger than L2: the step reads 2.3 GB; the decode pass evicts the prefill inputs",
+        },
+        "frac_of_nominal_bf16": pf_tflops_1 / NOMINAL_BF16_TFLOPS,
+        "roofline": {"bound": "tensor", "kernel": lib.kernel_name(0).replace("<D>", "<128>"),
+                     "achieved": pf_tflops_1, "peak": meas_tf, "unit": "TFLOP/s", "frac": pf_tflops_1 / meas_tf,
+                     "peak_source": f"{peak_src} bf16 burst (cuBLAS)", "traffic": args.prefill_traffic},
+        "decode": {
+            "value": dec_value, "unit": "GB/s", "ms_per_call": dec_avg_s * 1e3,
+            "algorithmic_bytes_per_call": dec_bytes,
+            "frac_of_nominal_hbm": dec_gbs_1 / NOMINAL_HBM_GBS,
+            "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<128,4> + decode_combine_kernel<128>",
+                         "achieved": dec_gbs_1, "peak": meas_bw, "unit": "GB/s", "frac": dec_gbs_1 / meas_bw,
+                         "peak_source": f"{peak_src} copy bandwidth", "traffic": args.decode_traffic},
+            "e2e": dec_e2e and {
+                "value": world * dec_bytes / (dec_e2e["ms"] * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": dec_e2e["h2d"], "d2h_bytes_per_step": dec_e2e["d2h"]},
+        },
+        "e2e": {"value": world * pf_flops / (e2e["ms"] * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+        "gates": gates,
+        "gpu_launches": 3 * K,
+        "kernels": {"prefill": lib.kernel_name(0), "decode": [lib.kernel_name(1), lib.kernel_name(2)]},
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    return line
+
+
+def time_prefill(lib, w, dev, stream, peaks, reps=20, warm=5):
+    import torch
+
+    q = synth.normal_bf16_torch(w.seed, synth.STREAM_Q, (w.B, w.Nq, w.Hq, w.d), dev)
+    k = synth.normal_bf16_torch(w.seed, synth.STREAM_K, (w.B, w.Nkv, w.Hkv, w.d), dev)
+    v = synth.normal_bf16_torch(w.seed, synth.STREAM_V, (w.B, w.Nkv, w.Hkv, w.d), dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(warm):
+        lib.attn_fwd(q, k, v, scale=w.scale, causal=w.causal, out=o, lse=lse)
+    ms = []
+    for _ in range(reps):
+        flush.fill_(1)  # 256 MiB write: L2 holds none of the inputs when the kernel starts
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        lib.attn_fwd(q, k, v, scale=w.scale, causal=w.causal, out=o, lse=lse)
+        b.record(stream)
+        b.synchronize()
+        ms.append(a.elapsed_time(b))
+    med = float(np.median(ms))
+    tf = w.flops / (med * 1e-3) / 1e12
+    return {"ms": med, "tflops": tf, "frac_of_measured": tf / peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]),
+            "frac_of_nominal": tf / NOMINAL_BF16_TFLOPS}
+
+
+def e2e_prefill(lib, P, q, k, v, stream, n):
+    """Host (pinned) -> device copies, attn_fwd, device -> host copies of O and LSE, per step."""
+    import torch
+
+    hq = q.cpu().pin_memory()
+    hk = k.cpu().pin_memory()
+    hv = v.cpu().pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ho = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    hl = torch.empty((P.B, P.Hq, P.Nq), dtype=torch.float32).pin_memory()
+
+    def one():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        o, lse = lib.attn_fwd(dq, dk, dv, scale=P.scale, causal=P.causal)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        one()
+    b.record(stream)
+    b.synchronize()
+    h2d = 3 * q.numel() * 2
+    d2h = q.numel() * 2 + P.B * P.Hq * P.Nq * 4
+    return {"ms": a.elapsed_time(b) / n, "h2d": h2d, "d2h": d2h}
+
+
+def e2e_decode(lib, Dw, dq, kc, vc, lens_np, stream, n):
+    """The decode call with its whole KV cache copied from pinned host memory every step."""
+    import torch
+
+    try:
+        hq = dq.cpu().pin_memory()
+        hk = kc.cpu().pin_memory()
+        hv = vc.cpu().pin_memory()
+    except RuntimeError:
+        return None
+    hl = torch.from_numpy(lens_np).pin_memory()
+    d_q, d_k, d_v = torch.empty_like(dq), torch.empty_like(kc), torch.empty_like(vc)
+    d_l = torch.empty(len(lens_np), dtype=torch.int32, device=dq.device)
+    ho = torch.empty(dq.shape, dtype=dq.dtype).pin_memory()
+    hls = torch.empty((Dw.B, Dw.Hq), dtype=torch.float32).pin_memory()
+
+    def one():
+        d_q.copy_(hq, non_blocking=True)
+        d_k.copy_(hk, non_blocking=True)
+        d_v.copy_(hv, non_blocking=True)
+        d_l.copy_(hl, non_blocking=True)
+        o, lse = lib.attn_decode_splitkv(d_q, d_k, d_v, d_l, scale=Dw.scale)
+        ho.copy_(o, non_blocking=True)
+        hls.copy_(lse, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        one()
+    b.record(stream)
+    b.synchronize()
+    h2d = (dq.numel() + kc.numel() + vc.numel()) * 2 + len(lens_np) * 4
+    d2h = dq.numel() * 2 + Dw.B * Dw.Hq * 4
+    out = {"ms": a.elapsed_time(b) / n, "h2d": h2d, "d2h": d2h}
+    del hk, hv, d_k, d_v
+    torch.cuda.empty_cache()
+    return out
+
+
+# ------------------------------------------------------------------------------------------------
+# reference arm: the CPU oracle, timed as it stands
+# ------------------------------------------------------------------------------------------------
+_HEAD_CACHE = {}
+
+
+def _rows_inputs(w: synth.Prefill, b: int, h: int, i0: int, m: int):
+    """Query rows [i0, i0+m) of head (b, h) and the keys they can see (all keys when not causal)."""
+    if (b, h) not in _HEAD_CACHE:
+        _HEAD_CACHE[(b, h)] = _head_inputs(w, b, h)
+    q, k, v = _HEAD_CACHE[(b, h)]
+    nk = min(w.Nkv, i0 + m + (w.Nkv - w.Nq)) if w.causal else w.Nkv
+    # with Nq = m and Nkv = nk, the bottom-right causal mask gives row r the keys j <= r + i0 + (Nkv - Nq)
+    flops = 4.0 * w.d * (sum(min(nk, i + 1 + (w.Nkv - w.Nq)) for i in range(i0, i0 + m)) if w.causal else m * nk)
+    return q[:, i0:i0 + m], k[:, :nk], v[:, :nk], flops
+
+
+def run_reference(args, world, rank):
+    """The CPU oracle as it stands, on bounded samples of the GPU arm's workloads, rank 0 only."""
+    import oracle
+
+    if rank != 0:
+        return None
+    P, Dw = synth.CAUSAL_2K, synth.DECODE
+    m = 64
+    blocks = [(b, h, i0) for (b, h) in ((0, 0), (1, 5), (2, 10), (3, 15)) for i0 in range(0, P.Nq, m)]
+    per_step = min(1.0, 100.0 / max(1, args.steps))  # keeps K steps within a couple of minutes
+    cursor = 0
+
+    def one_step():
+        nonlocal cursor
+        fl, sp, n = 0.0, 0.0, 0
+        while n == 0 or sp < per_step:
+            b, h, i0 = blocks[(cursor * 7919) % len(blocks)]
+            cursor += 1
+            q, k, v, f = _rows_inputs(P, b, h, i0, m)
+            t0 = time.perf_counter()
+            oracle.attention(q, k, v, P.scale, P.causal)
+            sp += time.perf_counter() - t0
+            fl += f
+            n += 1
+        return fl, sp, n
+
+    for _ in range(args.warmup):
+        one_step()
+    flops, spent, nblk = 0.0, 0.0, 0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        f, sp, n = one_step()
+        flops += f
+        spent += sp
+        nblk += n
+    wall = time.perf_counter() - t0
+    value = flops / spent / 1e12
+    dv, dsample, _ = cpu_decode(Dw, min(8.0, max(2.0, args.cpu_budget / 2)))
+    cores = _blas_threads()
+    sample = (f"{nblk} blocks of {m} query rows (with the keys they see) of {P.name}, "
+              f"{spent:.1f} s of oracle time over {args.steps} steps")
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": wall * 1e3 / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic: seeded i.i.d. N(0,1) rounded to bf16",
+        "config": {"workload": P.name, "decode_workload": Dw.name,
+                   "parallelism": "CPU oracle on rank 0 only", "l2": "n/a (CPU)"},
+        "decode": {"value": dv, "unit": "GB/s", "sample": dsample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "gpu_launches": 0,
+    }
+
+
+def run_only(args):
+    """One kernel on one workload, K timed launches (for profiling runs and per-workload numbers)."""
+    import torch
+
+    import exact_io_aware_41_b200 as lib
+
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    peaks, src = _peaks()
+    if args.only == "prefill":
+        table = {w.name: w for w in synth.PREFILL_WORKLOADS}
+        w = table[args.workload] if args.workload else synth.CAUSAL_2K
+        q = synth.normal_bf16_torch(w.seed, synth.STREAM_Q, (w.B, w.Nq, w.Hq, w.d), dev)
+        k = synth.normal_bf16_torch(w.seed, synth.STREAM_K, (w.B, w.Nkv, w.Hkv, w.d), dev)
+        v = synth.normal_bf16_torch(w.seed, synth.STREAM_V, (w.B, w.Nkv, w.Hkv, w.d), dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+
+        def call():
+            lib.attn_fwd(q, k, v, scale=w.scale, causal=w.causal, out=o, lse=lse)
+        work, unit, name = w.flops / 1e12, "TFLOP/s", w.name
+    else:
+        w = synth.DECODE
+        lens_np = np.minimum(w.lengths(), args.decode_cap) if args.decode_cap else w.lengths()
+        cap = int(args.decode_cap or w.cap)
+        dq = synth.normal_bf16_torch(w.seed, synth.STREAM_Q, (w.B, w.Hq, w.d), dev)
+        kc = synth.normal_bf16_torch(w.seed, synth.STREAM_K, (w.B, cap, w.Hkv, w.d), dev)
+        vc = synth.normal_bf16_torch(w.seed, synth.STREAM_V, (w.B, cap, w.Hkv, w.d), dev)
+        lens = torch.from_numpy(lens_np.astype(np.int32)).to(dev)
+        do = torch.empty_like(dq)
+        dl = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+        ws = torch.empty(lib.attn_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.d, cap, args.chunk), dtype=torch.uint8,
+                         device=dev)
+
+        def call():
+            lib.attn_decode_splitkv(dq, kc, vc, lens, scale=w.scale, chunk=args.chunk, workspace=ws, out=do, lse=dl)
+        byts = int(lens_np.astype(np.int64).sum()) * w.Hkv * w.d * 4 + w.B * w.Hq * (w.d * 4 + 4)
+        work, unit, name = byts / 1e9, "GB/s", f"{w.name} (lengths capped at {cap})"
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()  # drop the generator's temporaries: only the workload stays on the device
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in evs:
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    med = float(np.median(ms))
+    err = lib.attn_get_last_error()
+    print(json.dumps({"only": args.only, "workload": name, "median_ms": med, "value": work / (med * 1e-3),
+                      "unit": unit, "steps": args.steps, "warmup": args.warmup, "device_error": err}), flush=True)
+    if err != lib.ATTN_OK:
+        raise SystemExit(1)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-gates", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e-decode", action="store_true")
+    ap.add_argument("--prefill-traffic", type=float, default=None,
+                    help="ncu dram bytes per prefill launch, when measured for the current kernel")
+    ap.add_argument("--decode-traffic", type=float, default=None)
+    ap.add_argument("--only", choices=("prefill", "decode"), default=None,
+                    help="time one kernel on one workload (profiling and per-workload numbers)")
+    ap.add_argument("--workload", default=None, help="prefill workload name for --only prefill")
+    ap.add_argument("--decode-cap", type=int, default=0, help="cap decode lengths/cache for --only decode")
+    ap.add_argument("--chunk", type=int, default=0, help="decode chunk for --only decode (0 = automatic)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.only:
+        run_only(args)
+        return
+    world, rank, local, dist = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, world, rank)
+        else:
+            line = run_ours(args, world, rank, local, dist)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
