@@ -3,7 +3,8 @@
 Argument marshalling only: every function below checks dtypes, shapes and devices of torch tensors,
 allocates outputs with torch when the caller passes none, and calls the entry point of the same name
 in ``libattn_b200.so``. All attention arithmetic runs in that library's CUDA kernels; there is no
-other code path. If the library is missing the import fails with a message saying how to build it.
+other code path. The library is loaded on first use; if it is missing, that first call raises ImportError saying
+how to build it.
 """
 from __future__ import annotations
 
@@ -56,15 +57,23 @@ def _load() -> ctypes.CDLL:
     return lib
 
 
-_lib = _load()
+_handle = None
+
+
+def lib_handle() -> ctypes.CDLL:
+    """The loaded library (loaded on first use; raises ImportError if it is not built)."""
+    global _handle
+    if _handle is None:
+        _handle = _load()
+    return _handle
 
 
 def status_string(code: int) -> str:
-    return _lib.attn_status_string(int(code)).decode()
+    return lib_handle().attn_status_string(int(code)).decode()
 
 
 def kernel_name(which: int) -> str | None:
-    r = _lib.attn_kernel_name(int(which))
+    r = lib_handle().attn_kernel_name(int(which))
     return None if r is None else r.decode()
 
 
@@ -107,18 +116,18 @@ def attn_fwd(q, k, v, scale: float | None = None, causal: bool = False, out=None
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
-    code = _lib.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv,
+    code = lib_handle().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv,
                          Nq, Nkv, d, float(scale), int(bool(causal)), _stream(stream))
     _check("attn_fwd", code)
     return out, lse
 
 
 def attn_decode_workspace_bytes(B: int, Hq: int, Hkv: int, d: int, Nkv_cap: int, chunk: int = 0) -> int:
-    return int(_lib.attn_decode_workspace_bytes(B, Hq, Hkv, d, Nkv_cap, chunk))
+    return int(lib_handle().attn_decode_workspace_bytes(B, Hq, Hkv, d, Nkv_cap, chunk))
 
 
 def attn_decode_default_chunk(B: int, Hkv: int, Nkv_cap: int) -> int:
-    return int(_lib.attn_decode_default_chunk(B, Hkv, Nkv_cap))
+    return int(lib_handle().attn_decode_default_chunk(B, Hkv, Nkv_cap))
 
 
 def attn_decode_splitkv(q, k_cache, v_cache, kv_lens, scale: float | None = None, chunk: int = 0,
@@ -145,7 +154,7 @@ def attn_decode_splitkv(q, k_cache, v_cache, kv_lens, scale: float | None = None
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    code = _lib.attn_decode_splitkv(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), kv_lens.data_ptr(), cap,
+    code = lib_handle().attn_decode_splitkv(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), kv_lens.data_ptr(), cap,
                                     out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, d, float(scale), int(chunk),
                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                     _stream(stream))
@@ -164,7 +173,7 @@ def attn_decode_combine(part_o, part_lse, out=None, lse=None, stream=None):
         out = torch.empty((rows, d), dtype=torch.bfloat16, device=part_o.device)
     if lse is None:
         lse = torch.empty((rows,), dtype=torch.float32, device=part_o.device)
-    code = _lib.attn_decode_combine(part_o.data_ptr(), part_lse.data_ptr(), rows, n_splits, d, out.data_ptr(),
+    code = lib_handle().attn_decode_combine(part_o.data_ptr(), part_lse.data_ptr(), rows, n_splits, d, out.data_ptr(),
                                     lse.data_ptr(), _stream(stream))
     _check("attn_decode_combine", code)
     return out, lse
@@ -172,8 +181,8 @@ def attn_decode_combine(part_o, part_lse, out=None, lse=None, stream=None):
 
 def attn_get_last_error() -> int:
     """Reads and clears the device error word (synchronises). Returns a status code."""
-    return int(_lib.attn_get_last_error())
+    return int(lib_handle().attn_get_last_error())
 
 
 def attn_selftest_bounded_wait(limit_us: int, stream=None) -> None:
-    _check("attn_selftest_bounded_wait", _lib.attn_selftest_bounded_wait(int(limit_us), _stream(stream)))
+    _check("attn_selftest_bounded_wait", lib_handle().attn_selftest_bounded_wait(int(limit_us), _stream(stream)))

@@ -75,7 +75,7 @@ def test_decode_workspace_sizing():
 def test_argument_errors_are_reported_before_any_launch(raw):
     import exact_io_aware_41_b200 as pkg
 
-    lib = pkg._lib
+    lib = pkg.lib_handle()
     p = 1 << 20  # aligned, never dereferenced: every call below fails validation first
     # null pointer
     assert lib.attn_fwd(0, p, p, p, p, 1, 2, 2, 16, 16, 64, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG
