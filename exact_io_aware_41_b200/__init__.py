@@ -21,6 +21,7 @@ ATTN_ERR_UNSUPPORTED = 2
 ATTN_ERR_WORKSPACE = 3
 ATTN_ERR_CUDA = 4
 ATTN_ERR_TIMEOUT = 5
+DECODE_STATIC_SCRATCH_BYTES = 48 << 20  # ATTN_DECODE_STATIC_SCRATCH_BYTES
 
 # Function name -> (restype, argtypes), mirroring include/attn.h.
 _P = ctypes.c_void_p
@@ -31,6 +32,7 @@ SIGNATURES = {
     "attn_decode_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
     "attn_decode_default_chunk": (_I, [_I, _I, _I]),
     "attn_decode_splitkv": (_I, [_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _F, _I, _P, ctypes.c_size_t, _P]),
+    "attn_decode_splitkv_static": (_I, [_P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "attn_decode_combine": (_I, [_P, _P, _I, _I, _I, _P, _P, _P]),
     "attn_get_last_error": (_I, []),
     "attn_status_string": (ctypes.c_char_p, [_I]),
@@ -159,6 +161,36 @@ def attn_decode_splitkv(q, k_cache, v_cache, kv_lens, scale: float | None = None
                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                                     _stream(stream))
     _check("attn_decode_splitkv", code)
+    return out, lse
+
+
+def attn_decode_splitkv_static(q, k_cache, v_cache, kv_lens, scale: float | None = None, chunk: int = 0, out=None,
+                               lse=None, stream=None):
+    """attn_decode_splitkv with its partials in the library's fixed device array (no workspace).
+
+    For callers that cannot allocate device scratch. Outputs are allocated here only when the caller
+    passes none; the library call itself allocates nothing. Calls that overlap on the GPU share the
+    array and race.
+    """
+    import torch
+
+    _bf16_cuda("q", q, 3)
+    _bf16_cuda("k_cache", k_cache, 4)
+    _bf16_cuda("v_cache", v_cache, 4)
+    if kv_lens.dtype != torch.int32 or not kv_lens.is_cuda or kv_lens.dim() != 1:
+        raise ValueError("kv_lens must be a 1-d int32 CUDA tensor")
+    B, Hq, d = q.shape
+    _, cap, Hkv, _ = k_cache.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    code = lib_handle().attn_decode_splitkv_static(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), kv_lens.data_ptr(),
+                                           cap, out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, d, float(scale),
+                                           int(chunk), _stream(stream))
+    _check("attn_decode_splitkv_static", code)
     return out, lse
 
 

@@ -94,6 +94,33 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
                                   size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Size of the fixed device array that attn_decode_splitkv_static keeps its partials in (48 MiB).
+ * The array belongs to the loaded library: every GPU that loads it holds these bytes until exit.
+ */
+#define ATTN_DECODE_STATIC_SCRATCH_BYTES (48u << 20)
+
+/*
+ * attn_decode_splitkv without a workspace argument, for callers that cannot allocate device
+ * memory: a plugin running inside a host runtime that owns all device memory and offers it no
+ * allocator, or a latency-critical loop that must not call cudaMalloc (it can synchronise the device
+ * and can fail under memory pressure). The pages have no counterpart to this entry point; it only
+ * changes where the per-split partials live.
+ *
+ * Arguments, result and arithmetic are those of attn_decode_splitkv. The caller still passes q, the
+ * caches, kv_lens, o and lse. The partials go to one file-scope device array of
+ * ATTN_DECODE_STATIC_SCRATCH_BYTES; nothing is allocated and no allocating routine is called.
+ *  - Sizes whose partials (see attn_decode_workspace_bytes) exceed that array are rejected with
+ *    ATTN_ERR_WORKSPACE before anything is enqueued; a larger chunk makes the partials smaller.
+ *  - The first call on each device looks up the array's device address on the current device
+ *    (cudaGetSymbolAddress) and caches it; make that first call before any stream capture.
+ *  - Every call shares the one array and it keeps the last call's partials. Calls that overlap on
+ *    the GPU (on different streams, or from different host threads without ordering) race on it.
+ */
+attn_status_t attn_decode_splitkv_static(const void* q, const void* k_cache, const void* v_cache,
+                                         const int32_t* kv_lens, int Nkv_cap, void* o, float* lse, int B,
+                                         int Hq, int Hkv, int d, float scale, int chunk, cudaStream_t stream);
+
+/*
  * The combine step on its own: merges n_splits partial states per row with
  *     LSE = log sum_s exp(lse_s),   O = sum_s exp(lse_s - LSE) * o_s
  * ("FlashAttention evolution", section 6). Partials with lse_s = -inf contribute nothing; a row
