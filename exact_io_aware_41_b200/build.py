@@ -1,7 +1,8 @@
 """Builds the C-ABI shared library ``libattn_b200.so`` in this package directory.
 
-nvcc compiles every source under ``csrc/`` for sm_100a only (``-gencode arch=compute_100a,
-code=sm_100a``) with relocatable device code, and links them into one shared object that exports
+nvcc compiles ``csrc/attn_lib.cu``, which includes every other source under ``csrc/``, as one
+translation unit for sm_100a only (``-gencode arch=compute_100a,code=sm_100a``) into one shared
+object that exports
 the ``extern "C"`` entry points declared in ``include/attn.h``. Run ``python -m
 exact_io_aware_41_b200.build`` (``--force`` rebuilds, ``--verbose`` prints ptxas resource usage).
 """
@@ -17,6 +18,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB_PATH = os.path.join(HERE, "libattn_b200.so")
+UNITY = os.path.join(HERE, "csrc", "attn_lib.cu")  # includes every other .cu under csrc/
 SOURCES = sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
 HEADERS = sorted(glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + glob.glob(os.path.join(HERE, "csrc", "*.h")) +
                  glob.glob(os.path.join(ROOT, "include", "*.h")))
@@ -40,8 +42,8 @@ def up_to_date() -> bool:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB_PATH
-    cmd = [_nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-rdc=true", "-shared", "-Xcompiler", "-fPIC",
-           "-I", os.path.join(ROOT, "include"), "-o", LIB_PATH + ".tmp", *SOURCES]
+    cmd = [_nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-shared", "-Xcompiler", "-fPIC",
+           "-I", os.path.join(ROOT, "include"), "-o", LIB_PATH + ".tmp", UNITY]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     res = subprocess.run(cmd, capture_output=True, text=True)

@@ -8,24 +8,6 @@
 
 namespace attn {
 
-__device__ unsigned int g_error_word = 0;
-
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                            uint64_t limit_ns) {
-  const uint64_t t0 = global_timer_ns();
-  for (;;) {
-#pragma unroll 1
-    for (int i = 0; i < 256; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (abort_flag != nullptr && *abort_flag) return false;
-    if (global_timer_ns() - t0 > limit_ns) {
-      atomicOr(&g_error_word, kErrTimeoutBit);
-      if (abort_flag != nullptr) *abort_flag = 1;
-      return false;
-    }
-  }
-}
-
 // One CTA waits on a barrier that is initialised for one arrival and never receives it.
 __global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns) {
   __shared__ uint64_t bar;
@@ -69,7 +51,7 @@ bool encode_tile_map(CUtensorMap* map, const void* base, int d, int heads, int r
   return r == CUDA_SUCCESS;
 }
 
-static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool is_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace attn
 
@@ -80,7 +62,7 @@ extern "C" {
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                        int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+  if (!is_aligned16(q) || !is_aligned16(k) || !is_aligned16(v) || !is_aligned16(o) || !is_aligned16(lse))
     return ATTN_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
@@ -103,7 +85,7 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
                                   int Nkv_cap, void* o, float* lse, int B, int Hq, int Hkv, int d, float scale,
                                   int chunk, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!q || !k_cache || !v_cache || !kv_lens || !o || !lse) return ATTN_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(lse) ||
+  if (!is_aligned16(q) || !is_aligned16(k_cache) || !is_aligned16(v_cache) || !is_aligned16(o) || !is_aligned16(lse) ||
       (reinterpret_cast<uintptr_t>(kv_lens) & 3u))
     return ATTN_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || Nkv_cap < 1 || Hq % Hkv != 0 || chunk < 0 || (chunk % 64) != 0)
@@ -114,7 +96,7 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
   if (chunk == 0) chunk = decode_default_chunk(B, Hkv, Nkv_cap);
   const long long n_splits = (Nkv_cap + (long long)chunk - 1) / chunk;
   const size_t need = decode_workspace(B, Hq, d, Nkv_cap, chunk);
-  if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  if (workspace == nullptr || !is_aligned16(workspace) || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
   if (Hkv > 65535 || B > 65535) return ATTN_ERR_UNSUPPORTED;
   float* po = static_cast<float*>(workspace);
   const size_t po_bytes = size_t(B) * Hq * n_splits * d * sizeof(float);
@@ -129,7 +111,7 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
 attn_status_t attn_decode_combine(const float* part_o, const float* part_lse, int rows, int n_splits, int d,
                                   void* o, float* lse, cudaStream_t stream) {
   if (!part_o || !part_lse || !o || !lse) return ATTN_ERR_INVALID_ARG;
-  if (!aligned16(part_o) || !aligned16(o) || (reinterpret_cast<uintptr_t>(part_lse) & 3u) ||
+  if (!is_aligned16(part_o) || !is_aligned16(o) || (reinterpret_cast<uintptr_t>(part_lse) & 3u) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return ATTN_ERR_INVALID_ARG;
   if (rows < 1 || n_splits < 1) return ATTN_ERR_INVALID_ARG;

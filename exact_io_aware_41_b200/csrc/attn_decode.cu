@@ -34,7 +34,7 @@ struct DecCfg {
   static constexpr int LPT = D / 8;                       // lanes per token row
   static constexpr int R = 32 / LPT;                      // token rows per warp-wide load
   static constexpr int U0 = LPT / G;
-  static constexpr int U = U0 < 1 ? 1 : (U0 > 8 ? 8 : U0);  // rows in flight per lane
+  static constexpr int U = U0 < 1 ? 1 : (U0 > 4 ? 4 : U0);  // rows in flight per lane
   static constexpr int NV = G * U;                        // partial sums per lane before reduction
   static constexpr int TPI = U * R;                       // tokens per warp iteration
   static constexpr int LOG_LPT = (LPT == 8) ? 3 : (LPT == 16) ? 4 : 5;
@@ -45,11 +45,11 @@ struct DecCfg {
 };
 
 template <int D, int G>
-__global__ void __launch_bounds__(kDecodeWarps * 32)
+__global__ void __launch_bounds__(kDecodeWarps * 32, 4)
     decode_split_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
                         const __nv_bfloat16* __restrict__ vc, const int32_t* __restrict__ kv_lens, int Nkv_cap,
-                        int Hkv, int chunk, int n_splits, float scale, float scale_log2,
-                        float* __restrict__ part_o, float* __restrict__ part_lse) {
+                        int Hkv, int chunk, int n_splits, float scale_log2, float* __restrict__ part_o,
+                        float* __restrict__ part_lse) {
   using C = DecCfg<D, G>;
   const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -68,20 +68,20 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     return;
   }
 
+  // the group's query rows, pre-scaled by scale*log2(e) (scores come out in log2 units)
+  __shared__ __align__(16) float sq[G][D];
+  for (int i = threadIdx.x; i < G * D / 8; i += blockDim.x) {
+    const int hh = i / (D / 8), e = (i % (D / 8)) * 8;
+    float f[8];
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(q + (row0 + hh) * D + e), f);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) sq[hh][e + k] = f[k] * scale_log2;
+  }
+  __syncthreads();
+
   const int sub = lane % C::LPT;   // which 8 elements of d this lane covers
   const int r = lane / C::LPT;     // which token row of a warp-wide load
   const int e0 = sub * 8;
-
-  // query rows of the group, 8 elements per lane, pre-scaled by scale*log2(e)
-  float qf[G][8];
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(q + (row0 + hh) * D + e0);
-    bf16x8_to_f32(raw, qf[hh]);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) qf[hh][i] *= scale_log2;
-  }
-
   const size_t tok_stride = size_t(Hkv) * D;  // elements between consecutive tokens
   const __nv_bfloat16* kbase = kc + (size_t(b) * Nkv_cap * Hkv + g) * D + e0;
   const __nv_bfloat16* vbase = vc + (size_t(b) * Nkv_cap * Hkv + g) * D + e0;
@@ -101,43 +101,45 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
     for (int i = 0; i < 8; ++i) acc[hh][i] = 0.f;
   }
 
-  uint4 kr[C::U], vr[C::U];
-  auto load_rows = [&](int tb, uint4* kd, uint4* vd) {
+  // Rows of a warp iteration: token tb + u*R + r for u < U. Loads past t_end are skipped (zeros).
+  auto load_rows = [&](const __nv_bfloat16* base, int tb, uint4* dst) {
 #pragma unroll
     for (int uu = 0; uu < C::U; ++uu) {
       const int t = tb + uu * C::R + r;
-      if (t < t_end) {
-        kd[uu] = __ldcs(reinterpret_cast<const uint4*>(kbase + size_t(t) * tok_stride));
-        vd[uu] = __ldcs(reinterpret_cast<const uint4*>(vbase + size_t(t) * tok_stride));
-      } else {
-        kd[uu] = make_uint4(0, 0, 0, 0);
-        vd[uu] = make_uint4(0, 0, 0, 0);
-      }
+      dst[uu] = (t < t_end) ? __ldcs(reinterpret_cast<const uint4*>(base + size_t(t) * tok_stride))
+                            : make_uint4(0, 0, 0, 0);
     }
   };
 
   const int stride = kDecodeWarps * C::TPI;
   int tb = t_begin + warp * C::TPI;
-  if (tb < t_end) load_rows(tb, kr, vr);
+  uint4 kr[C::U], vr[C::U];
+  if (tb < t_end) load_rows(kbase, tb, kr);
   for (; tb < t_end; tb += stride) {
-    uint4 kn[C::U], vn[C::U];
-    const int tn = tb + stride;
-    if (tn < t_end) load_rows(tn, kn, vn);
+    // V rows of this iteration are only needed after the softmax: issue them first
+    load_rows(vbase, tb, vr);
 
     // ---- partial dot products: val[u*G + head] over this lane's 8 elements
     float val[C::NV];
 #pragma unroll
-    for (int uu = 0; uu < C::U; ++uu) {
-      float kf[8];
-      bf16x8_to_f32(kr[uu], kf);
+    for (int hh = 0; hh < G; ++hh) {
+      const float4 qa = *reinterpret_cast<const float4*>(&sq[hh][e0]);
+      const float4 qb = *reinterpret_cast<const float4*>(&sq[hh][e0 + 4]);
+      const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
+      for (int uu = 0; uu < C::U; ++uu) {
+        float kf[8];
+        bf16x8_to_f32(kr[uu], kf);
         float a = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) a = fmaf(qf[hh][i], kf[i], a);
+        for (int i = 0; i < 8; ++i) a = fmaf(qv[i], kf[i], a);
         val[uu * G + hh] = a;
       }
     }
+    // the K registers are free again: start the next iteration's K rows now
+    const int tn = tb + stride;
+    if (tn < t_end) load_rows(kbase, tn, kr);
+
     // ---- reduce across the LPT lanes of a token row: reduce-scatter while >1 value, then all-reduce
     {
       int cnt = C::NV;
@@ -202,11 +204,6 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
         for (int i = 0; i < 8; ++i) acc[hh][i] = fmaf(pp, vf[i], acc[hh][i]);
       }
     }
-#pragma unroll
-    for (int uu = 0; uu < C::U; ++uu) {
-      kr[uu] = kn[uu];
-      vr[uu] = vn[uu];
-    }
   }
 
   // ---- warp-level totals: acc over the R token rows, l over the distinct (u, r) lanes of a head
@@ -258,61 +255,113 @@ __global__ void __launch_bounds__(kDecodeWarps * 32)
   }
 }
 
-// One warp per output row: LSE = log sum_s exp(lse_s), O = sum_s exp(lse_s - LSE) o_s.
+// One CTA per output row; each thread owns EPT consecutive elements of d. The partial LSEs are
+// reduced first, the live splits are compacted into a list in shared memory, and the partial
+// outputs are accumulated with four independent loads in flight per thread.
+// LSE = log sum_s exp(lse_s), O = sum_s exp(lse_s - LSE) o_s.
 template <int D>
-__global__ void __launch_bounds__(128)
+struct CombCfg {
+  static constexpr int NT = D <= 128 ? 32 : 64;  // threads per row
+  static constexpr int EPT = D / NT;             // elements per thread (2 or 4)
+};
+
+template <int EPT>
+struct VecF;
+template <>
+struct VecF<2> {
+  using T = float2;
+  static __device__ __forceinline__ void fma(float w, const float* src, float* acc) {
+    const float2 v = *reinterpret_cast<const float2*>(src);
+    acc[0] = fmaf(w, v.x, acc[0]);
+    acc[1] = fmaf(w, v.y, acc[1]);
+  }
+};
+template <>
+struct VecF<4> {
+  static __device__ __forceinline__ void fma(float w, const float* src, float* acc) {
+    const float4 v = *reinterpret_cast<const float4*>(src);
+    acc[0] = fmaf(w, v.x, acc[0]);
+    acc[1] = fmaf(w, v.y, acc[1]);
+    acc[2] = fmaf(w, v.z, acc[2]);
+    acc[3] = fmaf(w, v.w, acc[3]);
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(CombCfg<D>::NT)
     decode_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse, int rows,
                           int n_splits, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
-  constexpr int EPL = D / 32;  // elements per lane
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 4 + warp;
-  if (row >= rows) return;
+  constexpr int NT = CombCfg<D>::NT, EPT = CombCfg<D>::EPT;
+  extern __shared__ float s_w[];  // [n_splits] weights of the live splits, then their indices
+  __shared__ float red[NT / 32];
+  __shared__ int n_live;
+  int* live = reinterpret_cast<int*>(s_w + n_splits);
+  const int row = blockIdx.x;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const float* pl = part_lse + size_t(row) * n_splits;
   float mx = -INFINITY;
-  for (int s = lane; s < n_splits; s += 32) mx = fmaxf(mx, pl[s]);
+  for (int s = t; s < n_splits; s += NT) mx = fmaxf(mx, pl[s]);
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  float acc[EPL];
+  if (lane == 0) red[warp] = mx;
+  if (t == 0) n_live = 0;
+  __syncthreads();
+  mx = red[0];
 #pragma unroll
-  for (int i = 0; i < EPL; ++i) acc[i] = 0.f;
-  float z = 0.f;
-  if (mx != -INFINITY) {
-    for (int s = 0; s < n_splits; ++s) {
-      const float ls = pl[s];
-      if (ls == -INFINITY) continue;
-      const float w = expf(ls - mx);
-      z += w;
-      const float* po = part_o + (size_t(row) * n_splits + s) * D + lane * EPL;
-#pragma unroll
-      for (int i = 0; i < EPL; i += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(po + i);
-        acc[i] = fmaf(w, v.x, acc[i]);
-        acc[i + 1] = fmaf(w, v.y, acc[i + 1]);
-        acc[i + 2] = fmaf(w, v.z, acc[i + 2]);
-        acc[i + 3] = fmaf(w, v.w, acc[i + 3]);
-      }
+  for (int w = 1; w < NT / 32; ++w) mx = fmaxf(mx, red[w]);
+  // weights and the compacted list of live splits (the order does not matter for the sums)
+  for (int s = t; s < n_splits; s += NT) {
+    const float ls = pl[s];
+    if (ls != -INFINITY) {
+      const int k = atomicAdd(&n_live, 1);
+      live[k] = s;
+      s_w[k] = expf(ls - mx);
     }
   }
-  const float inv = (z > 0.f) ? 1.0f / z : 0.f;
-  __nv_bfloat16* orow = o + size_t(row) * D + lane * EPL;
+  __syncthreads();
+  const int nl = n_live;
+  float acc[4][EPT];
 #pragma unroll
-  for (int i = 0; i < EPL; i += 2) {
-    const uint32_t pk = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
-    *reinterpret_cast<uint32_t*>(orow + i) = pk;
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) acc[i][e] = 0.f;
+  float z = 0.f;
+  const float* po = part_o + size_t(row) * n_splits * D + t * EPT;
+  int k = 0;
+  for (; k + 4 <= nl; k += 4) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float w = s_w[k + i];
+      z += w;
+      VecF<EPT>::fma(w, po + size_t(live[k + i]) * D, acc[i]);
+    }
   }
-  if (lane == 0) lse[row] = (z > 0.f) ? mx + logf(z) : -INFINITY;
+  for (; k < nl; ++k) {
+    const float w = s_w[k];
+    z += w;
+    VecF<EPT>::fma(w, po + size_t(live[k]) * D, acc[0]);
+  }
+  const float inv = (z > 0.f) ? 1.0f / z : 0.f;
+  __nv_bfloat16* orow = o + size_t(row) * D + t * EPT;
+#pragma unroll
+  for (int e = 0; e < EPT; e += 2) {
+    const float a0 = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
+    const float a1 = (acc[0][e + 1] + acc[1][e + 1]) + (acc[2][e + 1] + acc[3][e + 1]);
+    *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16x2(a0 * inv, a1 * inv);
+  }
+  if (t == 0) lse[row] = (z > 0.f) ? mx + logf(z) : -INFINITY;
 }
 
 // ---------------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------------
 int decode_default_chunk(int B, int Hkv, int Nkv_cap) {
-  // aim for ~8 live CTAs per SM if every sequence were full, in multiples of 64 tokens, at most 512
+  // aim for ~8 live CTAs per SM if every sequence were full, in multiples of 64 tokens, at most 1024
   const long long total = (long long)B * Hkv * Nkv_cap;
   long long c = total / (148LL * 8);
   c = (c + 63) / 64 * 64;
   if (c < 64) c = 64;
-  if (c > 512) c = 512;
+  if (c > 1024) c = 1024;
   return int(c);
 }
 
@@ -330,7 +379,7 @@ static attn_status_t launch_split(const void* q, const void* kc, const void* vc,
   dim3 grid(n_splits, Hkv, B);
   decode_split_kernel<D, G><<<grid, kDecodeWarps * 32, 0, stream>>>(
       reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(kc),
-      reinterpret_cast<const __nv_bfloat16*>(vc), lens, cap, Hkv, chunk, n_splits, scale,
+      reinterpret_cast<const __nv_bfloat16*>(vc), lens, cap, Hkv, chunk, n_splits,
       scale * 1.4426950408889634f, po, pl);
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
 }
@@ -362,12 +411,23 @@ attn_status_t decode_split_dispatch(const void* q, const void* kc, const void* v
 
 attn_status_t decode_combine_dispatch(const float* po, const float* pl, int rows, int n_splits, int d, void* o,
                                       float* lse, cudaStream_t st) {
-  const dim3 grid((rows + 3) / 4);
+  const dim3 grid(rows);
   __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(o);
+  const size_t sm = size_t(n_splits) * (sizeof(float) + sizeof(int));  // weights + live split list
+  if (sm > 200 * 1024) return ATTN_ERR_UNSUPPORTED;
   switch (d) {
-    case 64: decode_combine_kernel<64><<<grid, 128, 0, st>>>(po, pl, rows, n_splits, ob, lse); break;
-    case 128: decode_combine_kernel<128><<<grid, 128, 0, st>>>(po, pl, rows, n_splits, ob, lse); break;
-    case 256: decode_combine_kernel<256><<<grid, 128, 0, st>>>(po, pl, rows, n_splits, ob, lse); break;
+    case 64:
+      if (sm > 48 * 1024) cudaFuncSetAttribute(decode_combine_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm));
+      decode_combine_kernel<64><<<grid, CombCfg<64>::NT, sm, st>>>(po, pl, rows, n_splits, ob, lse);
+      break;
+    case 128:
+      if (sm > 48 * 1024) cudaFuncSetAttribute(decode_combine_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm));
+      decode_combine_kernel<128><<<grid, CombCfg<128>::NT, sm, st>>>(po, pl, rows, n_splits, ob, lse);
+      break;
+    case 256:
+      if (sm > 48 * 1024) cudaFuncSetAttribute(decode_combine_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm));
+      decode_combine_kernel<256><<<grid, CombCfg<256>::NT, sm, st>>>(po, pl, rows, n_splits, ob, lse);
+      break;
     default: return ATTN_ERR_UNSUPPORTED;
   }
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);

@@ -42,8 +42,6 @@ cudaError_t scratch_address(void** out) {
   return cudaSuccess;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 }  // namespace attn
 
@@ -54,7 +52,8 @@ extern "C" attn_status_t attn_decode_splitkv_static(const void* q, const void* k
                                                      int Hq, int Hkv, int d, float scale, int chunk,
                                                      cudaStream_t stream) {
   if (!q || !k_cache || !v_cache || !kv_lens || !o || !lse) return ATTN_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(lse) ||
+  if (!is_aligned16(q) || !is_aligned16(k_cache) || !is_aligned16(v_cache) || !is_aligned16(o) ||
+      !is_aligned16(lse) ||
       (reinterpret_cast<uintptr_t>(kv_lens) & 3u))
     return ATTN_ERR_INVALID_ARG;
   if (B < 1 || Hq < 1 || Hkv < 1 || Nkv_cap < 1 || Hq % Hkv != 0 || chunk < 0 || (chunk % 64) != 0)

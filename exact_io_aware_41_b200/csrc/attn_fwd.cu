@@ -34,6 +34,38 @@ namespace attn {
 // Running-max slack before O is rescaled, in log2 units: P entries stay <= 2^TAU.
 constexpr float kRescaleTau = 8.0f;
 
+// Columns (per 128 keys) whose exponential is evaluated on the FMA pipe instead of the exp unit,
+// in tiles without masked keys (the exp unit and the tensor cores need about the same number of
+// cycles per tile at d = 128, so moving part of the exponentials frees the bottleneck).
+#ifndef ATTN_EMU_COLS
+#define ATTN_EMU_COLS 0
+#endif
+constexpr int kEmuCols = ATTN_EMU_COLS;
+static_assert(kEmuCols % 8 == 0 && kEmuCols >= 0 && kEmuCols <= 128, "emulated column count");
+
+// 2^x for a pair, on the FMA pipe (x <= 128). Cody-Waite range reduction: x = n + f with
+// n = round(x) (the 1.5 * 2^23 addition rounds to an integer held in the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients come from a relative-error
+// Remez fit (csrc/fit_exp2_poly.py, max relative error 7.5e-5); 2^n is added to the exponent
+// field. Inputs below -125 are clamped there (2^-125 instead of a smaller value).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f, c2 = 0.2426111251115799f,
+                  c3 = 0.0551716685295105f;
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);
+  float2 q = ffma2(make_float2(c3, c3), f, make_float2(c2, c2));
+  q = ffma2(q, f, make_float2(c1, c1));
+  q = ffma2(q, f, make_float2(c0, c0));
+  float2 out;
+  out.x = __int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23));
+  out.y = __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23));
+  return out;
+}
+
 template <int D>
 struct FwdCfg {
   static constexpr int BM = 128;                        // query rows per tile (TMEM lanes)
@@ -51,6 +83,8 @@ struct FwdCfg {
   static constexpr int STAGES = (D == 128 || D == 256) ? 4 : 8;
   static constexpr int NSMWG = (NQT == 2) ? 2 : 1;      // softmax warpgroups
   static constexpr int THREADS = 128 * (1 + NSMWG);
+  static constexpr int HALF_PAIRS = BN / 4;             // bf16 pairs (TMEM columns) of P per half tile
+  static constexpr int PV_KH = BN / 32;                 // PV k-steps (16 keys) per half tile
   // TMEM columns (fp32 each): two S slots, then one O accumulator per query tile.
   static constexpr int S_COL0 = 0;
   static constexpr int S_COL1 = BN;
@@ -58,7 +92,8 @@ struct FwdCfg {
   static constexpr int O_COL1 = 2 * BN + D;
   static constexpr int TMEM_COLS = 512;
   static_assert(2 * BN + NQT * D <= TMEM_COLS, "tensor memory budget");
-  static constexpr int NBARS = 1 + 2 * STAGES + 2 + 2 + NQT + 1;
+  // q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done, o_final[2], drain[2]
+  static constexpr int NBARS = 1 + 2 * STAGES + 2 + 2 + 1 + 2 + 2;
   static constexpr int SMEM_DATA = NQT * Q_TILE_BYTES + STAGES * KV_TILE_BYTES;
   // Pad small-d configurations so only one CTA (and one 512-column TMEM allocation) fits per SM.
   static constexpr int SMEM_MIN = 120 * 1024;
@@ -66,6 +101,15 @@ struct FwdCfg {
   static constexpr int SMEM_BYTES = SMEM_BYTES_RAW > SMEM_MIN ? SMEM_BYTES_RAW : SMEM_MIN;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
+
+// Signals an mbarrier once per warp after the warp's tcgen05.st have completed: each lane waits
+// for its own stores and fences them, the warp syncs, and one lane arrives (barrier count = 4 warps).
+__device__ __forceinline__ void warp_publish_tmem_stores(uint64_t* bar, int lane) {
+  tmem_st_wait();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
 
 template <int D>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
@@ -80,11 +124,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   uint64_t* q_full = bars;
   uint64_t* kv_full = q_full + 1;
   uint64_t* kv_empty = kv_full + C::STAGES;
-  uint64_t* s_full = kv_empty + C::STAGES;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = p_full + 2;
-  uint64_t* drain = o_done + C::NQT;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* s_full = kv_empty + C::STAGES;  // [slot]: S = Q K^T landed in TMEM
+  uint64_t* p_full = s_full + 2;            // [slot]: P (bf16) of that slot is in TMEM
+  uint64_t* o_done = p_full + 2;            // one phase per PV (single-tile path: O rescale needs PV_{j-1})
+  uint64_t* o_final = o_done + 1;           // [tile] one phase: every MMA of the tile is done
+  uint64_t* drain = o_final + 2;            // [tile] error path: MMAs in flight have finished
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -92,10 +137,17 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   const uint64_t T = args.timeout_ns;
 
   // ---- unit of work ------------------------------------------------------------------------
-  const int BH = args.B * args.Hq;
+  // Heads are taken in groups whose K/V fit comfortably in L2 (group size chosen on the host), so
+  // the CTAs running together share K/V; inside a group the units go heaviest first (all heads'
+  // last query block, then the one before, ...), the longest-processing-time order for causal.
   const int u = blockIdx.x;
-  const int qblk = args.n_qblk - 1 - u / BH;  // heaviest causal blocks first
-  const int bh = u % BH;
+  const int BH = args.B * args.Hq;
+  const int per_group = args.heads_per_group * args.n_qblk;
+  const int grp = u / per_group;
+  const int r_in = u % per_group;
+  const int gh = min(args.heads_per_group, BH - grp * args.heads_per_group);  // heads in this group
+  const int bh = grp * args.heads_per_group + r_in % gh;
+  const int qblk = args.n_qblk - 1 - r_in / gh;
   const int b = bh / args.Hq;
   const int h = bh % args.Hq;
   const int g = h / args.group;
@@ -117,10 +169,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 4);  // one arrival per softmax warp
     }
-    for (int i = 0; i < C::NQT; ++i) mbar_init(&o_done[i], 1);
-    mbar_init(drain, 1);
+    mbar_init(o_done, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&o_final[i], 1);
+      mbar_init(&drain[i], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -137,13 +192,50 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // With two softmax warpgroups the 128 control threads give registers to the 256 softmax threads:
+  // 128 * 88 + 256 * 200 = 62464 <= 384 * 168 (the launch allocation). Each role changes its budget
+  // at the top of its own branch so the new limit covers all of that role's code.
+  constexpr bool kSplitRegs = (C::NQT == 2);
+
+  // ---- MMA issue helpers (used by whichever thread issues a tile's MMAs) ----------------------
+  constexpr uint32_t idesc_qk = idesc_bf16_f32(128, C::BN, 0, 0);
+  constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+  // Only the start-address field (bits 0-13, 16-byte units) differs between the descriptors of one
+  // operand, so each base descriptor is built once and the k-step offsets are added to it.
+  // Shared-memory addresses stay below 2^18, so the field never carries into its neighbour.
+  const uint64_t dQ = smem_desc(smem_u32(sQ), 16, 8 * C::ROWB, C::LAYOUT);
+  const uint64_t dK = smem_desc(smem_u32(sKV), 16, 8 * C::ROWB, C::LAYOUT);
+  const uint64_t dV = smem_desc(smem_u32(sKV), C::KV_CHUNK_BYTES, 8 * C::ROWB, C::LAYOUT);
+  // S[slot] = Q_qt K^T : A = Q tile (K-major), B = K tile (K-major), k-steps of 16 along d.
+  auto issue_qk = [&](int qt, int s_col, int stage) {
+    const uint64_t a0 = dQ + uint64_t((qt * C::Q_TILE_BYTES) >> 4);
+    const uint64_t b0 = dK + uint64_t((stage * C::KV_TILE_BYTES) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t ao = (kk / C::KPC) * C::Q_CHUNK_BYTES + (kk % C::KPC) * 32;
+      const uint32_t bo = (kk / C::KPC) * C::KV_CHUNK_BYTES + (kk % C::KPC) * 32;
+      umma_ss(tmem + s_col, a0 + (ao >> 4), b0 + (bo >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+    }
+  };
+  // O += P V over k-steps [k_from, k_to) of 16 keys: A = P (bf16, in TMEM over S), B = V tile read
+  // MN-major (N = d).
+  auto issue_pv = [&](int o_col, int p_col, int stage, bool accumulate, int k_from, int k_to) {
+    const uint64_t b0 = dV + uint64_t((stage * C::KV_TILE_BYTES) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < C::BN / 16; ++kk) {
+      if (kk < k_from || kk >= k_to) continue;
+      umma_ts(tmem + o_col, tmem + p_col + kk * 8, b0 + uint64_t((kk * 16 * C::ROWB) >> 4), idesc_pv,
+              (accumulate || kk > 0) ? 1u : 0u);
+    }
+  };
+  // K/V ring positions: K_j at 2j, V_j at 2j + 1.
+  auto kv_slot = [](int pos) { return pos % C::STAGES; };
+  auto kv_phase = [](int pos) { return uint32_t((pos / C::STAGES) & 1); };
 
   if (warp == 0) {
     // ================================ TMA producer ================================
+    if (kSplitRegs) regs_dec<88>();
     if (lane == 0 && n_tiles > 0) {
-      int fills[C::STAGES];
-#pragma unroll
-      for (int s = 0; s < C::STAGES; ++s) fills[s] = 0;
       bool ok = true;
       mbar_arrive_expect_tx(q_full, C::NQT * C::Q_TILE_BYTES);
 #pragma unroll
@@ -152,7 +244,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         for (int c = 0; c < C::NCHUNK; ++c)
           tma_load_4d(sQ + qt * C::Q_TILE_BYTES + c * C::Q_CHUNK_BYTES, &tmQ, q_full, c * C::CHUNK, h,
                       q0 + qt * C::BM, b);
-      int pos = 0;
+      int pos = 0;  // ring position: K_j at 2j, V_j at 2j + 1
       for (int j = 0; j < n_tiles && ok; ++j) {
 #pragma unroll
         for (int kv = 0; kv < 2; ++kv, ++pos) {
@@ -168,55 +260,31 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           for (int c = 0; c < C::NCHUNK; ++c)
             tma_load_4d(sKV + s * C::KV_TILE_BYTES + c * C::KV_CHUNK_BYTES, m, &kv_full[s], c * C::CHUNK, g,
                         j * C::BN, b);
-          ++fills[s];
         }
       }
       if (!ok) {
         // Give the copies already in flight a bounded chance to land before the CTA exits.
         mbar_wait(q_full, 0, nullptr, 100000000ull);
-        for (int s = 0; s < C::STAGES; ++s)
-          if (fills[s] > 0) mbar_wait(&kv_full[s], (fills[s] - 1) & 1, nullptr, 100000000ull);
+        // ring positions [0, pos) were issued; slot s holds the fills at positions s, s + STAGES, ...
+        for (int s = 0; s < C::STAGES; ++s) {
+          const int fills = (pos - s + C::STAGES - 1) / C::STAGES;
+          if (fills > 0) mbar_wait(&kv_full[s], (fills - 1) & 1, nullptr, 100000000ull);
+        }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ================================ MMA issuer ================================
+    if (kSplitRegs) regs_dec<88>();
     if (lane == 0 && n_tiles > 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, C::BN, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t sQ_addr = smem_u32(sQ);
-      const uint32_t sKV_addr = smem_u32(sKV);
-      // S[slot] = Q_qt K^T : A = Q tile (K-major), B = K tile (K-major), k-steps of 16 along d.
-      auto issue_qk = [&](int qt, int s_col, int stage) {
-        const uint32_t a0 = sQ_addr + qt * C::Q_TILE_BYTES;
-        const uint32_t b0 = sKV_addr + stage * C::KV_TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ao = (kk / C::KPC) * C::Q_CHUNK_BYTES + (kk % C::KPC) * 32;
-          const uint32_t bo = (kk / C::KPC) * C::KV_CHUNK_BYTES + (kk % C::KPC) * 32;
-          umma_ss(tmem + s_col, smem_desc(a0 + ao, 16, 8 * C::ROWB, C::LAYOUT),
-                  smem_desc(b0 + bo, 16, 8 * C::ROWB, C::LAYOUT), idesc_qk, kk > 0 ? 1u : 0u);
-        }
-      };
-      // O_qt += P V : A = P (bf16, in TMEM over S), B = V tile read MN-major (N = d), k-steps of 16 keys.
-      auto issue_pv = [&](int o_col, int p_col, int stage, bool accumulate) {
-        const uint32_t b0 = sKV_addr + stage * C::KV_TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk) {
-          umma_ts(tmem + o_col, tmem + p_col + kk * 8,
-                  smem_desc(b0 + kk * 16 * C::ROWB, C::KV_CHUNK_BYTES, 8 * C::ROWB, C::LAYOUT), idesc_pv,
-                  (accumulate || kk > 0) ? 1u : 0u);
-        }
-      };
-      auto kv_slot = [&](int pos) { return pos % C::STAGES; };
-      auto kv_phase = [&](int pos) { return uint32_t((pos / C::STAGES) & 1); };
+      // K/V tiles and Q arrive by TMA (complete_tx on the mbarrier): the MMAs may read them once
+      // the barrier phase is observed. P is written to TMEM by the softmax threads' tcgen05.st, so
+      // observing p_full is followed by tcgen05.fence::after_thread_sync before the PV MMAs.
       bool ok = mbar_wait(q_full, 0, abort_flag, T);
-      tc_fence_after();
       if (C::NQT == 2) {
-        // Ring order: K_0, V_0, K_1, V_1, ...  (K_j at position 2j, V_j at 2j + 1)
+        // Two query tiles, one S slot each: QK(0,0) QK(1,0) | PV(0,j) QK(0,j+1) PV(1,j) QK(1,j+1) | ...
         if (ok) ok = mbar_wait(&kv_full[kv_slot(0)], kv_phase(0), abort_flag, T);
         if (ok) {
-          tc_fence_after();
           issue_qk(0, C::S_COL0, kv_slot(0));
           umma_commit(&s_full[0]);
           issue_qk(1, C::S_COL1, kv_slot(0));
@@ -228,16 +296,16 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           const bool nxt = j + 1 < n_tiles;
           ok = mbar_wait(&kv_full[kv_slot(pv_pos)], kv_phase(pv_pos), abort_flag, T);
           if (ok && nxt) ok = mbar_wait(&kv_full[kv_slot(pk_pos)], kv_phase(pk_pos), abort_flag, T);
-          if (!ok) break;
-          tc_fence_after();
 #pragma unroll
           for (int qt = 0; qt < 2; ++qt) {
+            if (!ok) break;
             const int s_col = qt ? C::S_COL1 : C::S_COL0;
             ok = mbar_wait(&p_full[qt], j & 1, abort_flag, T);
             if (!ok) break;
             tc_fence_after();
-            issue_pv(qt ? C::O_COL1 : C::O_COL0, s_col, kv_slot(pv_pos), j > 0);
-            umma_commit(&o_done[qt]);
+            issue_pv(qt ? C::O_COL1 : C::O_COL0, s_col, kv_slot(pv_pos), j > 0, 0, C::BN / 16);
+            // P of this tile is consumed by the PV MMAs above before this QK overwrites the slot:
+            // MMAs issued by one thread execute in issue order.
             if (nxt) {
               issue_qk(qt, s_col, kv_slot(pk_pos));
               umma_commit(&s_full[qt]);
@@ -252,7 +320,6 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         for (int j = 0; j < 2 && j < n_tiles && ok; ++j) {
           ok = mbar_wait(&kv_full[kv_slot(2 * j)], kv_phase(2 * j), abort_flag, T);
           if (!ok) break;
-          tc_fence_after();
           issue_qk(0, j ? C::S_COL1 : C::S_COL0, kv_slot(2 * j));
           umma_commit(&s_full[j]);
           umma_commit(&kv_empty[kv_slot(2 * j)]);
@@ -264,29 +331,35 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           if (ok) ok = mbar_wait(&p_full[slot], (j >> 1) & 1, abort_flag, T);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(C::O_COL0, s_col, kv_slot(2 * j + 1), j > 0);
-          umma_commit(&o_done[0]);
+          issue_pv(C::O_COL0, s_col, kv_slot(2 * j + 1), j > 0, 0, C::BN / 16);
+          umma_commit(o_done);
           umma_commit(&kv_empty[kv_slot(2 * j + 1)]);
           if (j + 2 < n_tiles) {
             const int kp = 2 * (j + 2);
             ok = mbar_wait(&kv_full[kv_slot(kp)], kv_phase(kp), abort_flag, T);
             if (!ok) break;
-            tc_fence_after();
             issue_qk(0, s_col, kv_slot(kp));
             umma_commit(&s_full[slot]);
             umma_commit(&kv_empty[kv_slot(kp)]);
           }
         }
       }
-      if (!ok) {
+      // o_final arrives once every MMA above has completed (one barrier per tile, both signalled).
+      if (ok) {
+        umma_commit(&o_final[0]);
+        if (C::NQT == 2) umma_commit(&o_final[1]);
+      } else {
         // Let the MMAs already issued finish before tensor memory is released.
-        umma_commit(drain);
-        mbar_wait(drain, 0, nullptr, 100000000ull);
+        umma_commit(&drain[0]);
+        mbar_wait(&drain[0], 0, nullptr, 100000000ull);
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    if (kSplitRegs) regs_dec<88>();
+  } else {
     // ================================ softmax warpgroups ================================
+    if (kSplitRegs) regs_inc<200>();
     const int wg = (warp - 4) >> 2;
     const int wq = warp & 3;             // warp within its warpgroup: TMEM lanes 32*wq .. 32*wq+31
     const int row = wq * 32 + lane;      // query row within the tile = TMEM lane
@@ -298,19 +371,22 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const float c = args.scale_log2;
     // last key visible to this row (any key index <= lim is visible); rows past Nq are padding
     const int lim = args.causal ? min(args.Nkv - 1, q_row + diag) : args.Nkv - 1;
+    // every lane waits; the warp continues only if all of them saw the phase (tcgen05.ld/st below are
+    // warp-collective, so a partial give-up must not split the warp)
+    auto wait_warp = [&](uint64_t* bar, uint32_t ph) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, ph, abort_flag, T));
+    };
 
     float m_ref = -INFINITY;  // reference max (raw-score units) of the exponentials in l and O
     float l = 0.f;            // running row sum of exp2(c * (s - m_ref))
-    bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      const int slot = (C::NQT == 2) ? qt : (j & 1);
-      const uint32_t ph = (C::NQT == 2) ? uint32_t(j & 1) : uint32_t((j >> 1) & 1);
-      const uint32_t s_addr = lane_addr + (slot ? C::S_COL1 : C::S_COL0);
-      if (!mbar_wait(&s_full[slot], ph, abort_flag, T)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
+
+    // One S tile -> P. Reads S from TMEM, masks, updates the running max (rescaling O in TMEM only
+    // when the max grew by more than TAU), and writes P = 2^(c*s - c*m_ref) as bf16 over the first
+    // BN/2 columns of the slot (two per 32-bit column; the S values it replaces are already in
+    // registers) in two halves, calling publish(half) after each half is stored. Pairs go through
+    // the packed FMA pipe; the exponential uses the exp unit (MUFU.EX2) or, for the last kEmuCols
+    // columns of tiles without masked keys, the FMA-pipe polynomial. Returns false if a wait gave up.
+    auto softmax_tile = [&](int j, uint32_t s_addr, auto&& publish) -> bool {
       uint32_t r[C::BN];
 #pragma unroll
       for (int cc = 0; cc < C::BN / 32; ++cc) tmem_ld32(s_addr + cc * 32, r + cc * 32);
@@ -326,9 +402,21 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         for (int i = 0; i < C::BN; ++i)
           if (kbase + i > lim) r[i] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
+      // row max: eight independent chains of 3-input max, then a short tree
+      float mx;
+      {
+        constexpr int Q8 = C::BN / 8;
+        float m8[8];
 #pragma unroll
-      for (int i = 0; i < C::BN; ++i) mx = fmaxf(mx, __uint_as_float(r[i]));
+        for (int k = 0; k < 8; ++k) {
+          float a = __uint_as_float(r[k * Q8]);
+#pragma unroll
+          for (int i = 1; i + 1 < Q8; i += 2)
+            a = fmax3(a, __uint_as_float(r[k * Q8 + i]), __uint_as_float(r[k * Q8 + i + 1]));
+          m8[k] = (Q8 % 2 == 0) ? fmaxf(a, __uint_as_float(r[k * Q8 + Q8 - 1])) : a;
+        }
+        mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+      }
       const float m_new = fmaxf(m_ref, mx);
       // true when the max moved by more than TAU (also on the first live tile: -inf -> finite)
       const bool need = (m_new - m_ref) * c > kRescaleTau;
@@ -338,11 +426,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         l *= alpha;
         if (j > 0) {
           if (C::NQT == 1) {
-            // PV_{j-1} must have landed in O before it is rescaled
-            if (!mbar_wait(&o_done[0], (j - 1) & 1, abort_flag, T)) {
-              ok = false;
-              break;
-            }
+            // PV_{j-1} must have landed in O before it is rescaled. (With two query tiles S_j is
+            // committed after PV_{j-1} of the same tile, so it has landed already.)
+            if (!wait_warp(o_done, (j - 1) & 1)) return false;
             tc_fence_after();
           }
 #pragma unroll 1
@@ -359,23 +445,60 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         }
       }
       const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
-      float rs0 = 0.f, rs1 = 0.f;
-      uint32_t p[C::BN / 2];
+      const float2 c2 = make_float2(c, c);
+      const float2 nmc2 = make_float2(-mc, -mc);
+      float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+      constexpr int EMU_FROM = (C::BN - kEmuCols * C::BN / 128) / 2;  // first emulated pair
+      const bool emu = kEmuCols > 0 && !need_mask;
 #pragma unroll
-      for (int i = 0; i < C::BN / 2; ++i) {
-        const float p0 = ex2(fmaf(__uint_as_float(r[2 * i]), c, -mc));
-        const float p1 = ex2(fmaf(__uint_as_float(r[2 * i + 1]), c, -mc));
-        rs0 += p0;
-        rs1 += p1;
-        p[i] = pack_bf16x2(p0, p1);
+      for (int half = 0; half < 2; ++half) {
+        uint32_t p[C::HALF_PAIRS];
+#pragma unroll
+        for (int i2 = 0; i2 < C::HALF_PAIRS; ++i2) {
+          const int i = half * C::HALF_PAIRS + i2;
+          const float2 x = ffma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nmc2);
+          float2 e;
+          if (i >= EMU_FROM && emu) {
+            e = exp2_poly2(x);
+          } else {
+            e.x = ex2(x.x);
+            e.y = ex2(x.y);
+          }
+          acc4[i & 3] = fadd2(acc4[i & 3], e);
+          p[i2] = pack_bf16x2(e.x, e.y);
+        }
+        if (C::HALF_PAIRS == 32)
+          tmem_st32(s_addr + half * C::HALF_PAIRS, p);
+        else
+          tmem_st16(s_addr + half * C::HALF_PAIRS, p);
+        publish(half);
       }
-      l += rs0 + rs1;
-      // P overwrites the first BN/2 columns of this S slot (two bf16 per 32-bit column)
-#pragma unroll
-      for (int cc = 0; cc < C::BN / 64; ++cc) tmem_st32(s_addr + cc * 32, p + cc * 32);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[slot]);
+      const float2 s01 = fadd2(acc4[0], acc4[1]);
+      const float2 s23 = fadd2(acc4[2], acc4[3]);
+      const float2 s = fadd2(s01, s23);
+      l += s.x + s.y;
+      return true;
+    };
+
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      // two query tiles: one S slot per tile; one query tile: S alternates between the two slots
+      const int slot = (C::NQT == 2) ? qt : (j & 1);
+      const uint32_t ph = (C::NQT == 2) ? uint32_t(j & 1) : uint32_t((j >> 1) & 1);
+      if (!wait_warp(&s_full[slot], ph)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // P is published once both halves are stored
+      auto publish = [&](int half) {
+        if (half == 1) warp_publish_tmem_stores(&p_full[slot], lane);
+      };
+      if (!softmax_tile(j, lane_addr + (slot ? C::S_COL1 : C::S_COL0), publish)) {
+        ok = false;
+        break;
+      }
     }
 
     // ---- epilogue: O = acc / l (once), LSE = scale * m_ref + ln l -------------------------------
@@ -383,7 +506,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.o) +
                           ((size_t(b) * args.Nq + (valid ? q_row : 0)) * args.Hq + h) * D;
     if (n_tiles > 0 && ok) {
-      ok = mbar_wait(&o_done[qt], (n_tiles - 1) & 1, abort_flag, T);
+      ok = wait_warp(&o_final[qt], 0);
       tc_fence_after();
     }
     if (ok) {
@@ -459,6 +582,15 @@ static attn_status_t launch_fwd(const void* q, const void* k, const void* v, voi
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.timeout_ns = kWaitLimitNs;
+  // heads per L2 group: K/V of one kv head is read by every query head of its group and block; keep
+  // a group's K/V within ~48 MB of the 126 MB L2
+  {
+    const double kv_bytes_per_head = 2.0 * Nkv * D * 2 / double(Hq / Hkv);
+    long long gh = (long long)(48.0e6 / kv_bytes_per_head);
+    if (gh < 1) gh = 1;
+    if (gh > (long long)B * Hq) gh = (long long)B * Hq;
+    a.heads_per_group = int(gh);
+  }
   const long long units = (long long)a.n_qblk * B * Hq;
   if (units > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
   attn_fwd_kernel<D><<<dim3(unsigned(units)), dim3(C::THREADS), C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, a);

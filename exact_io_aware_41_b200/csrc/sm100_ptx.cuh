@@ -10,7 +10,8 @@
 namespace attn {
 
 // Device-wide error word, OR-ed by any CTA whose bounded wait gave up (see attn_get_last_error).
-extern __device__ unsigned int g_error_word;
+// Defined here: the library is compiled as one translation unit.
+__device__ unsigned int g_error_word = 0;
 
 enum : unsigned int {
   kErrTimeoutBit = 1u,
@@ -60,17 +61,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait on the phase with the given parity. Gives up after `limit_ns` of wall time, or as
-// soon as another role of the CTA has raised `abort_flag`; on giving up it records the timeout in
-// the device error word, raises the CTA abort flag and returns false.
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                            uint64_t limit_ns);
-
+// soon as another role of the CTA has raised `abort_flag` (may be null); on giving up it records
+// the timeout in the device error word, raises the CTA abort flag and returns false. Inline on
+// purpose: an out-of-line call would make every waiting role save its live registers.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
 #pragma unroll 1
-  for (int i = 0; i < 16; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, abort_flag, limit_ns);
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (abort_flag != nullptr && *abort_flag) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      atomicOr(&g_error_word, kErrTimeoutBit);
+      if (abort_flag != nullptr) *abort_flag = 1;
+      return false;
+    }
+  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -238,6 +247,55 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// 3-input maximum (sm_100a).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Packed fp32 pairs on the FMA pipe (sm_100a f32x2): one instruction for two lanes' worth of work.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(reinterpret_cast<uint64_t&>(d))
+      : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)),
+        "l"(reinterpret_cast<const uint64_t&>(c)));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("add.f32x2 %0, %1, %2;"
+      : "=l"(reinterpret_cast<uint64_t&>(d))
+      : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)));
+  return d;
+}
+
+// Named barrier over one warpgroup (128 threads): plain sync, and sync with an AND of a predicate.
+__device__ __forceinline__ void wg_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+__device__ __forceinline__ bool wg_all(bool v, int id) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(uint32_t(v)), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
+// Register budget changes for warp-specialised roles (counts must be multiples of 8).
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 }  // namespace attn
