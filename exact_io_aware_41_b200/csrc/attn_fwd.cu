@@ -26,6 +26,8 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <atomic>
+
 #include "attn_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -92,12 +94,15 @@ struct FwdCfg {
   static constexpr int O_COL1 = 2 * BN + D;
   static constexpr int TMEM_COLS = 512;
   static_assert(2 * BN + NQT * D <= TMEM_COLS, "tensor memory budget");
-  // q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done, o_final[2], drain[2]
-  static constexpr int NBARS = 1 + 2 * STAGES + 2 + 2 + 1 + 2 + 2;
+  // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done, o_final[2], drain,
+  // sched_full[SCHED], sched_empty[SCHED]
+  static constexpr int SCHED = 4;  // units the producer may claim ahead of the consumers
+  static constexpr int NBARS = 2 + 2 * STAGES + 2 + 2 + 1 + 2 + 1 + 2 * SCHED;
+  static constexpr int SCHED_CONSUMERS = 1 + 4 * NSMWG;  // MMA thread + one arrival per softmax warp
   static constexpr int SMEM_DATA = NQT * Q_TILE_BYTES + STAGES * KV_TILE_BYTES;
   // Pad small-d configurations so only one CTA (and one 512-column TMEM allocation) fits per SM.
   static constexpr int SMEM_MIN = 120 * 1024;
-  static constexpr int SMEM_BYTES_RAW = 1024 + SMEM_DATA + NBARS * 8 + 16;
+  static constexpr int SMEM_BYTES_RAW = 1024 + SMEM_DATA + NBARS * 8 + 16 + SCHED * 4;
   static constexpr int SMEM_BYTES = SMEM_BYTES_RAW > SMEM_MIN ? SMEM_BYTES_RAW : SMEM_MIN;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
@@ -111,6 +116,50 @@ __device__ __forceinline__ void warp_publish_tmem_stores(uint64_t* bar, int lane
   if (lane == 0) mbar_arrive(bar);
 }
 
+// Dynamic unit scheduling: a launch claims units from one slot of these counters (next unit, CTAs
+// finished). The host gives each launch the next of kSchedSlots slots; the last CTA of a launch to
+// finish returns the slot to zero, so launches that follow each other never see a live counter.
+constexpr int kSchedSlots = 256;
+__device__ unsigned int g_sched_next[kSchedSlots];
+__device__ unsigned int g_sched_done[kSchedSlots];
+
+// Units in issue order: heads grouped so a group's K/V fit comfortably in L2 (group size chosen on
+// the host) and, inside a group, heaviest first (every head's last query block, then the one
+// before, ...), the longest-processing-time order for causal masks.
+struct Unit {
+  int b, h, q0;
+  int n_tiles;   // K/V tiles the unit streams (the last query tile's count)
+  int n_tile0;   // K/V tiles the first query tile needs (fewer when the last one is above its diagonal)
+};
+
+template <int D>
+__device__ __forceinline__ Unit unit_at(const FwdArgs& a, int lin) {
+  using C = FwdCfg<D>;
+  const int BH = a.B * a.Hq;
+  const int per_group = a.heads_per_group * a.n_qblk;
+  const int grp = lin / per_group;
+  const int r_in = lin % per_group;
+  const int gh = min(a.heads_per_group, BH - grp * a.heads_per_group);  // heads in this group
+  const int bh = grp * a.heads_per_group + r_in % gh;
+  const int qblk = a.n_qblk - 1 - r_in / gh;
+  Unit u;
+  u.b = bh / a.Hq;
+  u.h = bh % a.Hq;
+  u.q0 = qblk * C::NQT * C::BM;
+  int kv_end = a.Nkv;
+  if (a.causal) {
+    const int q_last = min(u.q0 + C::NQT * C::BM, a.Nq) - 1;
+    kv_end = min(a.Nkv, q_last + (a.Nkv - a.Nq) + 1);
+  }
+  u.n_tiles = kv_end > 0 ? (kv_end + C::BN - 1) / C::BN : 0;
+  u.n_tile0 = u.n_tiles;
+  if (C::NQT == 2 && a.causal) {
+    const int end0 = min(a.Nkv, min(u.q0 + C::BM, a.Nq) - 1 + (a.Nkv - a.Nq) + 1);
+    u.n_tile0 = end0 > 0 ? (end0 + C::BN - 1) / C::BN : 0;
+  }
+  return u;
+}
+
 template <int D>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -121,48 +170,31 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + C::NQT * C::Q_TILE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + C::STAGES * C::KV_TILE_BYTES);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = q_full + 1;
+  uint64_t* q_full = bars;                  // one phase per unit: Q tiles landed
+  uint64_t* q_empty = q_full + 1;           // one phase per unit: every MMA reading Q is done
+  uint64_t* kv_full = q_empty + 1;
   uint64_t* kv_empty = kv_full + C::STAGES;
   uint64_t* s_full = kv_empty + C::STAGES;  // [slot]: S = Q K^T landed in TMEM
   uint64_t* p_full = s_full + 2;            // [slot]: P (bf16) of that slot is in TMEM
   uint64_t* o_done = p_full + 2;            // one phase per PV (single-tile path: O rescale needs PV_{j-1})
-  uint64_t* o_final = o_done + 1;           // [tile] one phase: every MMA of the tile is done
-  uint64_t* drain = o_final + 2;            // [tile] error path: MMAs in flight have finished
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 2);
+  uint64_t* o_final = o_done + 1;           // [tile] one phase per unit: every MMA of the unit is done
+  uint64_t* drain = o_final + 2;            // error path: MMAs in flight have finished
+  uint64_t* sched_full = drain + 1;         // [SCHED] the producer wrote the k-th unit index
+  uint64_t* sched_empty = sched_full + C::SCHED;  // [SCHED] every role read it
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sched_empty + C::SCHED);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* sched_unit = reinterpret_cast<volatile int*>(tmem_holder + 2);  // [SCHED]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint64_t T = args.timeout_ns;
-
-  // ---- unit of work ------------------------------------------------------------------------
-  // Heads are taken in groups whose K/V fit comfortably in L2 (group size chosen on the host), so
-  // the CTAs running together share K/V; inside a group the units go heaviest first (all heads'
-  // last query block, then the one before, ...), the longest-processing-time order for causal.
-  const int u = blockIdx.x;
-  const int BH = args.B * args.Hq;
-  const int per_group = args.heads_per_group * args.n_qblk;
-  const int grp = u / per_group;
-  const int r_in = u % per_group;
-  const int gh = min(args.heads_per_group, BH - grp * args.heads_per_group);  // heads in this group
-  const int bh = grp * args.heads_per_group + r_in % gh;
-  const int qblk = args.n_qblk - 1 - r_in / gh;
-  const int b = bh / args.Hq;
-  const int h = bh % args.Hq;
-  const int g = h / args.group;
-  const int q0 = qblk * C::NQT * C::BM;
+  const int total_units = args.B * args.Hq * args.n_qblk;
   const int diag = args.Nkv - args.Nq;  // key j visible to query i iff j <= i + diag
-  int kv_end = args.Nkv;
-  if (args.causal) {
-    const int q_last = min(q0 + C::NQT * C::BM, args.Nq) - 1;
-    kv_end = min(args.Nkv, q_last + diag + 1);
-  }
-  const int n_tiles = kv_end > 0 ? (kv_end + C::BN - 1) / C::BN : 0;
 
   // ---- set-up --------------------------------------------------------------------------------
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
@@ -170,11 +202,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);  // one arrival per softmax warp
+      mbar_init(&o_final[i], 1);
     }
     mbar_init(o_done, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&o_final[i], 1);
-      mbar_init(&drain[i], 1);
+    mbar_init(drain, 1);
+    for (int i = 0; i < C::SCHED; ++i) {
+      mbar_init(&sched_full[i], 1);
+      mbar_init(&sched_empty[i], C::SCHED_CONSUMERS);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -193,11 +227,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   // With two softmax warpgroups the 128 control threads give registers to the 256 softmax threads:
-  // 128 * 88 + 256 * 200 = 62464 <= 384 * 168 (the launch allocation). Each role changes its budget
+  // 128 * 104 + 256 * 192 = 62464 <= 384 * 168 (the launch allocation). Each role changes its budget
   // at the top of its own branch so the new limit covers all of that role's code.
   constexpr bool kSplitRegs = (C::NQT == 2);
 
-  // ---- MMA issue helpers (used by whichever thread issues a tile's MMAs) ----------------------
+  // ---- MMA issue helpers ------------------------------------------------------------------------
   constexpr uint32_t idesc_qk = idesc_bf16_f32(128, C::BN, 0, 0);
   constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
   // Only the start-address field (bits 0-13, 16-byte units) differs between the descriptors of one
@@ -217,54 +251,89 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       umma_ss(tmem + s_col, a0 + (ao >> 4), b0 + (bo >> 4), idesc_qk, kk > 0 ? 1u : 0u);
     }
   };
-  // O += P V over k-steps [k_from, k_to) of 16 keys: A = P (bf16, in TMEM over S), B = V tile read
-  // MN-major (N = d).
-  auto issue_pv = [&](int o_col, int p_col, int stage, bool accumulate, int k_from, int k_to) {
+  // O += P V over the tile's keys: A = P (bf16, in TMEM over S), B = V tile read MN-major (N = d),
+  // k-steps of 16 keys.
+  auto issue_pv = [&](int o_col, int p_col, int stage, bool accumulate) {
     const uint64_t b0 = dV + uint64_t((stage * C::KV_TILE_BYTES) >> 4);
 #pragma unroll
-    for (int kk = 0; kk < C::BN / 16; ++kk) {
-      if (kk < k_from || kk >= k_to) continue;
+    for (int kk = 0; kk < C::BN / 16; ++kk)
       umma_ts(tmem + o_col, tmem + p_col + kk * 8, b0 + uint64_t((kk * 16 * C::ROWB) >> 4), idesc_pv,
               (accumulate || kk > 0) ? 1u : 0u);
-    }
   };
-  // K/V ring positions: K_j at 2j, V_j at 2j + 1.
+  // K/V ring positions run on across units; inside a unit K_j is at base + 2j, V_j at base + 2j + 1.
   auto kv_slot = [](int pos) { return pos % C::STAGES; };
   auto kv_phase = [](int pos) { return uint32_t((pos / C::STAGES) & 1); };
 
+  // The k-th unit of this CTA as handed out by the producer (-1: no more units or a wait gave up).
+  // Every consumer role reads the slot and then arrives once (one thread for the MMA warp, lane 0
+  // of each softmax warp after the warp has read it).
+  auto next_unit = [&](int k, bool whole_warp) -> int {
+    const int slot = k % C::SCHED;
+    const uint32_t ph = uint32_t((k / C::SCHED) & 1);
+    bool seen = mbar_wait(&sched_full[slot], ph, abort_flag, T);
+    if (whole_warp) seen = __all_sync(0xffffffffu, seen);
+    if (!seen) return -1;
+    const int lin = sched_unit[slot];
+    if (whole_warp) __syncwarp();
+    if (!whole_warp || lane == 0) mbar_arrive(&sched_empty[slot]);
+    return lin;
+  };
+
   if (warp == 0) {
     // ================================ TMA producer ================================
-    if (kSplitRegs) regs_dec<88>();
-    if (lane == 0 && n_tiles > 0) {
+    if (kSplitRegs) regs_dec<104>();
+    if (lane == 0) {
       bool ok = true;
-      mbar_arrive_expect_tx(q_full, C::NQT * C::Q_TILE_BYTES);
+      int pos = 0;  // next ring position
+      int qc = 0;   // units loaded so far (phase of q_full / q_empty)
+      for (int k = 0; ok; ++k) {
+        // claim the next unit (longest first) and hand it to the other roles
+        const int slot = k % C::SCHED;
+        if (!mbar_wait(&sched_empty[slot], uint32_t(((k / C::SCHED) & 1) ^ 1), abort_flag, T)) {
+          ok = false;
+          break;
+        }
+        const unsigned claimed = atomicAdd(&g_sched_next[args.sched_slot], 1u);
+        const int lin = claimed < unsigned(total_units) ? int(claimed) : -1;
+        sched_unit[slot] = lin;
+        mbar_arrive(&sched_full[slot]);
+        if (lin < 0) break;
+        const Unit un = unit_at<D>(args, lin);
+        if (un.n_tiles == 0) continue;
+        const int g = un.h / args.group;
+        // Q of the previous unit must be consumed by all its MMAs before it is overwritten
+        if (qc > 0 && !mbar_wait(q_empty, (qc - 1) & 1, abort_flag, T)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(q_full, C::NQT * C::Q_TILE_BYTES);
 #pragma unroll
-      for (int qt = 0; qt < C::NQT; ++qt)
-#pragma unroll
-        for (int c = 0; c < C::NCHUNK; ++c)
-          tma_load_4d(sQ + qt * C::Q_TILE_BYTES + c * C::Q_CHUNK_BYTES, &tmQ, q_full, c * C::CHUNK, h,
-                      q0 + qt * C::BM, b);
-      int pos = 0;  // ring position: K_j at 2j, V_j at 2j + 1
-      for (int j = 0; j < n_tiles && ok; ++j) {
-#pragma unroll
-        for (int kv = 0; kv < 2; ++kv, ++pos) {
-          const int s = pos % C::STAGES;
-          const uint32_t ph = (pos / C::STAGES) & 1;
-          if (!mbar_wait(&kv_empty[s], ph ^ 1, abort_flag, T)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&kv_full[s], C::KV_TILE_BYTES);
-          const CUtensorMap* m = kv ? &tmV : &tmK;
+        for (int qt = 0; qt < C::NQT; ++qt)
 #pragma unroll
           for (int c = 0; c < C::NCHUNK; ++c)
-            tma_load_4d(sKV + s * C::KV_TILE_BYTES + c * C::KV_CHUNK_BYTES, m, &kv_full[s], c * C::CHUNK, g,
-                        j * C::BN, b);
+            tma_load_4d(sQ + qt * C::Q_TILE_BYTES + c * C::Q_CHUNK_BYTES, &tmQ, q_full, c * C::CHUNK, un.h,
+                        un.q0 + qt * C::BM, un.b);
+        ++qc;
+        for (int j = 0; j < un.n_tiles && ok; ++j) {
+#pragma unroll
+          for (int kv = 0; kv < 2; ++kv, ++pos) {
+            const int s = kv_slot(pos);
+            if (!mbar_wait(&kv_empty[s], kv_phase(pos) ^ 1, abort_flag, T)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&kv_full[s], C::KV_TILE_BYTES);
+            const CUtensorMap* m = kv ? &tmV : &tmK;
+#pragma unroll
+            for (int c = 0; c < C::NCHUNK; ++c)
+              tma_load_4d(sKV + s * C::KV_TILE_BYTES + c * C::KV_CHUNK_BYTES, m, &kv_full[s], c * C::CHUNK, g,
+                          j * C::BN, un.b);
+          }
         }
       }
       if (!ok) {
         // Give the copies already in flight a bounded chance to land before the CTA exits.
-        mbar_wait(q_full, 0, nullptr, 100000000ull);
+        if (qc > 0) mbar_wait(q_full, (qc - 1) & 1, nullptr, 100000000ull);
         // ring positions [0, pos) were issued; slot s holds the fills at positions s, s + STAGES, ...
         for (int s = 0; s < C::STAGES; ++s) {
           const int fills = (pos - s + C::STAGES - 1) / C::STAGES;
@@ -275,243 +344,286 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ================================ MMA issuer ================================
-    if (kSplitRegs) regs_dec<88>();
-    if (lane == 0 && n_tiles > 0) {
-      // K/V tiles and Q arrive by TMA (complete_tx on the mbarrier): the MMAs may read them once
-      // the barrier phase is observed. P is written to TMEM by the softmax threads' tcgen05.st, so
+    if (kSplitRegs) regs_dec<104>();
+    if (lane == 0) {
+      // K/V tiles and Q arrive by TMA (complete_tx on the mbarrier): the MMAs may read them once the
+      // barrier phase is observed. P is written to TMEM by the softmax threads' tcgen05.st, so
       // observing p_full is followed by tcgen05.fence::after_thread_sync before the PV MMAs.
-      bool ok = mbar_wait(q_full, 0, abort_flag, T);
-      if (C::NQT == 2) {
-        // Two query tiles, one S slot each: QK(0,0) QK(1,0) | PV(0,j) QK(0,j+1) PV(1,j) QK(1,j+1) | ...
-        if (ok) ok = mbar_wait(&kv_full[kv_slot(0)], kv_phase(0), abort_flag, T);
-        if (ok) {
-          issue_qk(0, C::S_COL0, kv_slot(0));
-          umma_commit(&s_full[0]);
-          issue_qk(1, C::S_COL1, kv_slot(0));
-          umma_commit(&s_full[1]);
-          umma_commit(&kv_empty[kv_slot(0)]);
-        }
-        for (int j = 0; j < n_tiles && ok; ++j) {
-          const int pv_pos = 2 * j + 1, pk_pos = 2 * j + 2;
-          const bool nxt = j + 1 < n_tiles;
-          ok = mbar_wait(&kv_full[kv_slot(pv_pos)], kv_phase(pv_pos), abort_flag, T);
-          if (ok && nxt) ok = mbar_wait(&kv_full[kv_slot(pk_pos)], kv_phase(pk_pos), abort_flag, T);
+      bool ok = true;
+      int pos = 0;    // ring position of the next K/V tile to consume
+      int qc = 0;     // units issued (phase of q_full)
+      int pc[2] = {0, 0};  // P tiles consumed per slot (phase of p_full)
+      int t_run = 0;  // single-tile path: S tiles issued so far (slot = t_run & 1)
+      for (int k = 0; ok; ++k) {
+        const int lin = next_unit(k, false);
+        if (lin < 0) break;
+        const Unit un = unit_at<D>(args, lin);
+        const int n = un.n_tiles;
+        if (n == 0) continue;
+        ok = mbar_wait(q_full, qc & 1, abort_flag, T);
+        ++qc;
+        const int base = pos;  // K_j at base + 2j, V_j at base + 2j + 1
+        if (C::NQT == 2) {
+          // Two query tiles, one S slot each: QK(0,0) QK(1,0) | PV(0,j) QK(0,j+1) PV(1,j) QK(1,j+1) | ...
+          if (ok) ok = mbar_wait(&kv_full[kv_slot(base)], kv_phase(base), abort_flag, T);
+          // a causal unit's first query tile may need one K/V tile fewer than the second
+          const int nt[2] = {un.n_tile0, n};
+          if (ok) {
 #pragma unroll
-          for (int qt = 0; qt < 2; ++qt) {
-            if (!ok) break;
-            const int s_col = qt ? C::S_COL1 : C::S_COL0;
-            ok = mbar_wait(&p_full[qt], j & 1, abort_flag, T);
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv(qt ? C::O_COL1 : C::O_COL0, s_col, kv_slot(pv_pos), j > 0, 0, C::BN / 16);
-            // P of this tile is consumed by the PV MMAs above before this QK overwrites the slot:
-            // MMAs issued by one thread execute in issue order.
-            if (nxt) {
-              issue_qk(qt, s_col, kv_slot(pk_pos));
+            for (int qt = 0; qt < 2; ++qt) {
+              if (nt[qt] == 0) continue;
+              issue_qk(qt, qt ? C::S_COL1 : C::S_COL0, kv_slot(base));
               umma_commit(&s_full[qt]);
             }
+            umma_commit(&kv_empty[kv_slot(base)]);
           }
-          if (!ok) break;
-          umma_commit(&kv_empty[kv_slot(pv_pos)]);
-          if (nxt) umma_commit(&kv_empty[kv_slot(pk_pos)]);
-        }
-      } else {
-        // One query tile, S alternating between two slots: QK_0, QK_1, PV_0, QK_2, PV_1, QK_3, ...
-        for (int j = 0; j < 2 && j < n_tiles && ok; ++j) {
-          ok = mbar_wait(&kv_full[kv_slot(2 * j)], kv_phase(2 * j), abort_flag, T);
-          if (!ok) break;
-          issue_qk(0, j ? C::S_COL1 : C::S_COL0, kv_slot(2 * j));
-          umma_commit(&s_full[j]);
-          umma_commit(&kv_empty[kv_slot(2 * j)]);
-        }
-        for (int j = 0; j < n_tiles && ok; ++j) {
-          const int slot = j & 1;
-          const int s_col = slot ? C::S_COL1 : C::S_COL0;
-          ok = mbar_wait(&kv_full[kv_slot(2 * j + 1)], kv_phase(2 * j + 1), abort_flag, T);
-          if (ok) ok = mbar_wait(&p_full[slot], (j >> 1) & 1, abort_flag, T);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(C::O_COL0, s_col, kv_slot(2 * j + 1), j > 0, 0, C::BN / 16);
-          umma_commit(o_done);
-          umma_commit(&kv_empty[kv_slot(2 * j + 1)]);
-          if (j + 2 < n_tiles) {
-            const int kp = 2 * (j + 2);
-            ok = mbar_wait(&kv_full[kv_slot(kp)], kv_phase(kp), abort_flag, T);
+          for (int j = 0; j < n && ok; ++j) {
+            const int pv_pos = base + 2 * j + 1, pk_pos = base + 2 * j + 2;
+            const bool nxt = j + 1 < n;
+            ok = mbar_wait(&kv_full[kv_slot(pv_pos)], kv_phase(pv_pos), abort_flag, T);
+            if (ok && nxt) ok = mbar_wait(&kv_full[kv_slot(pk_pos)], kv_phase(pk_pos), abort_flag, T);
+#pragma unroll
+            for (int qt = 0; qt < 2; ++qt) {
+              if (!ok) break;
+              if (j >= nt[qt]) continue;
+              const int s_col = qt ? C::S_COL1 : C::S_COL0;
+              ok = mbar_wait(&p_full[qt], pc[qt] & 1, abort_flag, T);
+              if (!ok) break;
+              ++pc[qt];
+              tc_fence_after();
+              issue_pv(qt ? C::O_COL1 : C::O_COL0, s_col, kv_slot(pv_pos), j > 0);
+              // P of this tile is consumed by the PV MMAs above before this QK overwrites the slot:
+              // MMAs issued by one thread execute in issue order.
+              if (j + 1 < nt[qt]) {
+                issue_qk(qt, s_col, kv_slot(pk_pos));
+                umma_commit(&s_full[qt]);
+              }
+            }
             if (!ok) break;
-            issue_qk(0, s_col, kv_slot(kp));
-            umma_commit(&s_full[slot]);
-            umma_commit(&kv_empty[kv_slot(kp)]);
+            umma_commit(&kv_empty[kv_slot(pv_pos)]);
+            if (nxt) umma_commit(&kv_empty[kv_slot(pk_pos)]);
           }
+          pos = base + 2 * n;
+        } else {
+          // One query tile, S alternating between two slots: QK_0, QK_1, PV_0, QK_2, PV_1, QK_3, ...
+          const int t0 = t_run;
+          for (int j = 0; j < 2 && j < n && ok; ++j) {
+            ok = mbar_wait(&kv_full[kv_slot(base + 2 * j)], kv_phase(base + 2 * j), abort_flag, T);
+            if (!ok) break;
+            issue_qk(0, ((t0 + j) & 1) ? C::S_COL1 : C::S_COL0, kv_slot(base + 2 * j));
+            umma_commit(&s_full[(t0 + j) & 1]);
+            umma_commit(&kv_empty[kv_slot(base + 2 * j)]);
+          }
+          for (int j = 0; j < n && ok; ++j) {
+            const int t = t0 + j;
+            const int slot = t & 1;
+            const int s_col = slot ? C::S_COL1 : C::S_COL0;
+            ok = mbar_wait(&kv_full[kv_slot(base + 2 * j + 1)], kv_phase(base + 2 * j + 1), abort_flag, T);
+            if (ok) ok = mbar_wait(&p_full[slot], (t >> 1) & 1, abort_flag, T);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(C::O_COL0, s_col, kv_slot(base + 2 * j + 1), j > 0);
+            umma_commit(o_done);
+            umma_commit(&kv_empty[kv_slot(base + 2 * j + 1)]);
+            if (j + 2 < n) {
+              const int kp = base + 2 * (j + 2);
+              ok = mbar_wait(&kv_full[kv_slot(kp)], kv_phase(kp), abort_flag, T);
+              if (!ok) break;
+              issue_qk(0, s_col, kv_slot(kp));
+              umma_commit(&s_full[slot]);
+              umma_commit(&kv_empty[kv_slot(kp)]);
+            }
+          }
+          t_run = t0 + n;
+          pos = base + 2 * n;
         }
-      }
-      // o_final arrives once every MMA above has completed (one barrier per tile, both signalled).
-      if (ok) {
+        if (!ok) break;
+        // every MMA of this unit done: Q may be reloaded, O may be read (one o_final per tile)
+        umma_commit(q_empty);
         umma_commit(&o_final[0]);
         if (C::NQT == 2) umma_commit(&o_final[1]);
-      } else {
+      }
+      if (!ok) {
         // Let the MMAs already issued finish before tensor memory is released.
-        umma_commit(&drain[0]);
-        mbar_wait(&drain[0], 0, nullptr, 100000000ull);
+        umma_commit(drain);
+        mbar_wait(drain, 0, nullptr, 100000000ull);
       }
     }
     __syncwarp();
   } else if (warp < 4) {
-    if (kSplitRegs) regs_dec<88>();
+    if (kSplitRegs) regs_dec<104>();
   } else {
     // ================================ softmax warpgroups ================================
-    if (kSplitRegs) regs_inc<200>();
+    if (kSplitRegs) regs_inc<192>();
     const int wg = (warp - 4) >> 2;
     const int wq = warp & 3;             // warp within its warpgroup: TMEM lanes 32*wq .. 32*wq+31
     const int row = wq * 32 + lane;      // query row within the tile = TMEM lane
     const int qt = (C::NQT == 2) ? wg : 0;
-    const int q_first = q0 + qt * C::BM;
-    const int q_row = q_first + row;
     const uint32_t lane_addr = tmem + (uint32_t(wq * 32) << 16);
     const uint32_t o_col = qt ? C::O_COL1 : C::O_COL0;
     const float c = args.scale_log2;
-    // last key visible to this row (any key index <= lim is visible); rows past Nq are padding
-    const int lim = args.causal ? min(args.Nkv - 1, q_row + diag) : args.Nkv - 1;
     // every lane waits; the warp continues only if all of them saw the phase (tcgen05.ld/st below are
     // warp-collective, so a partial give-up must not split the warp)
     auto wait_warp = [&](uint64_t* bar, uint32_t ph) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, ph, abort_flag, T));
     };
 
-    float m_ref = -INFINITY;  // reference max (raw-score units) of the exponentials in l and O
-    float l = 0.f;            // running row sum of exp2(c * (s - m_ref))
-
-    // One S tile -> P. Reads S from TMEM, masks, updates the running max (rescaling O in TMEM only
-    // when the max grew by more than TAU), and writes P = 2^(c*s - c*m_ref) as bf16 over the first
-    // BN/2 columns of the slot (two per 32-bit column; the S values it replaces are already in
-    // registers) in two halves, calling publish(half) after each half is stored. Pairs go through
-    // the packed FMA pipe; the exponential uses the exp unit (MUFU.EX2) or, for the last kEmuCols
-    // columns of tiles without masked keys, the FMA-pipe polynomial. Returns false if a wait gave up.
-    auto softmax_tile = [&](int j, uint32_t s_addr, auto&& publish) -> bool {
-      uint32_t r[C::BN];
-#pragma unroll
-      for (int cc = 0; cc < C::BN / 32; ++cc) tmem_ld32(s_addr + cc * 32, r + cc * 32);
-      tmem_ld_wait();
-#pragma unroll
-      for (int cc = 0; cc < C::BN / 32; ++cc) tmem_reg_fence32(r + cc * 32);
-
-      const int kbase = j * C::BN;
-      // warp-uniform: does any key of this tile fall outside some row's visible range?
-      const bool need_mask = (kbase + C::BN > args.Nkv) || (args.causal && kbase + C::BN - 1 > q_first + diag);
-      if (need_mask) {
-#pragma unroll
-        for (int i = 0; i < C::BN; ++i)
-          if (kbase + i > lim) r[i] = __float_as_uint(-INFINITY);
-      }
-      // row max: eight independent chains of 3-input max, then a short tree
-      float mx;
-      {
-        constexpr int Q8 = C::BN / 8;
-        float m8[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          float a = __uint_as_float(r[k * Q8]);
-#pragma unroll
-          for (int i = 1; i + 1 < Q8; i += 2)
-            a = fmax3(a, __uint_as_float(r[k * Q8 + i]), __uint_as_float(r[k * Q8 + i + 1]));
-          m8[k] = (Q8 % 2 == 0) ? fmaxf(a, __uint_as_float(r[k * Q8 + Q8 - 1])) : a;
-        }
-        mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-      }
-      const float m_new = fmaxf(m_ref, mx);
-      // true when the max moved by more than TAU (also on the first live tile: -inf -> finite)
-      const bool need = (m_new - m_ref) * c > kRescaleTau;
-      if (__any_sync(0xffffffffu, need)) {
-        const float alpha = need ? ex2((m_ref - m_new) * c) : 1.0f;
-        if (need) m_ref = m_new;
-        l *= alpha;
-        if (j > 0) {
-          if (C::NQT == 1) {
-            // PV_{j-1} must have landed in O before it is rescaled. (With two query tiles S_j is
-            // committed after PV_{j-1} of the same tile, so it has landed already.)
-            if (!wait_warp(o_done, (j - 1) & 1)) return false;
-            tc_fence_after();
-          }
-#pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            tmem_ld32(lane_addr + o_col + cc * 32, o);
-            tmem_ld_wait();
-            tmem_reg_fence32(o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(lane_addr + o_col + cc * 32, o);
-          }
-          tmem_st_wait();
-        }
-      }
-      const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
-      const float2 c2 = make_float2(c, c);
-      const float2 nmc2 = make_float2(-mc, -mc);
-      float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                        make_float2(0.f, 0.f)};
-      constexpr int EMU_FROM = (C::BN - kEmuCols * C::BN / 128) / 2;  // first emulated pair
-      const bool emu = kEmuCols > 0 && !need_mask;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t p[C::HALF_PAIRS];
-#pragma unroll
-        for (int i2 = 0; i2 < C::HALF_PAIRS; ++i2) {
-          const int i = half * C::HALF_PAIRS + i2;
-          const float2 x = ffma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nmc2);
-          float2 e;
-          if (i >= EMU_FROM && emu) {
-            e = exp2_poly2(x);
-          } else {
-            e.x = ex2(x.x);
-            e.y = ex2(x.y);
-          }
-          acc4[i & 3] = fadd2(acc4[i & 3], e);
-          p[i2] = pack_bf16x2(e.x, e.y);
-        }
-        if (C::HALF_PAIRS == 32)
-          tmem_st32(s_addr + half * C::HALF_PAIRS, p);
-        else
-          tmem_st16(s_addr + half * C::HALF_PAIRS, p);
-        publish(half);
-      }
-      const float2 s01 = fadd2(acc4[0], acc4[1]);
-      const float2 s23 = fadd2(acc4[2], acc4[3]);
-      const float2 s = fadd2(s01, s23);
-      l += s.x + s.y;
-      return true;
-    };
-
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      // two query tiles: one S slot per tile; one query tile: S alternates between the two slots
-      const int slot = (C::NQT == 2) ? qt : (j & 1);
-      const uint32_t ph = (C::NQT == 2) ? uint32_t(j & 1) : uint32_t((j >> 1) & 1);
-      if (!wait_warp(&s_full[slot], ph)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // P is published once both halves are stored
-      auto publish = [&](int half) {
-        if (half == 1) warp_publish_tmem_stores(&p_full[slot], lane);
-      };
-      if (!softmax_tile(j, lane_addr + (slot ? C::S_COL1 : C::S_COL0), publish)) {
-        ok = false;
-        break;
-      }
-    }
+    int sc = 0;     // S tiles consumed by this warpgroup (two tiles: phase of s_full[qt])
+    int t_run = 0;  // single-tile path: S tiles consumed so far (slot = t_run & 1)
+    int uc = 0;     // units with keys finished (phase of o_final)
+    for (int k = 0; ok; ++k) {
+      const int lin = next_unit(k, true);
+      if (lin < 0) break;
+      const Unit un = unit_at<D>(args, lin);
+      const int q_first = un.q0 + qt * C::BM;
+      const int q_row = q_first + row;
+      // last key visible to this row (any key index <= lim is visible); rows past Nq are padding
+      const int lim = args.causal ? min(args.Nkv - 1, q_row + diag) : args.Nkv - 1;
+      float m_ref = -INFINITY;  // reference max (raw-score units) of the exponentials in l and O
+      float l = 0.f;            // running row sum of exp2(c * (s - m_ref))
 
-    // ---- epilogue: O = acc / l (once), LSE = scale * m_ref + ln l -------------------------------
-    const bool valid = q_row < args.Nq;
-    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.o) +
-                          ((size_t(b) * args.Nq + (valid ? q_row : 0)) * args.Hq + h) * D;
-    if (n_tiles > 0 && ok) {
-      ok = wait_warp(&o_final[qt], 0);
-      tc_fence_after();
-    }
-    if (ok) {
-      const float inv = (l > 0.f) ? 1.0f / l : 0.f;
-      if (n_tiles > 0) {
+      const int my_tiles = (qt == 0) ? un.n_tile0 : un.n_tiles;
+      for (int j = 0; j < my_tiles; ++j) {
+        // two query tiles: one S slot per tile; one query tile: S alternates between the two slots
+        const int slot = (C::NQT == 2) ? qt : (t_run & 1);
+        const uint32_t ph = (C::NQT == 2) ? uint32_t(sc & 1) : uint32_t((t_run >> 1) & 1);
+        if (!wait_warp(&s_full[slot], ph)) {
+          ok = false;
+          break;
+        }
+        ++sc;
+        ++t_run;
+        tc_fence_after();
+        const uint32_t s_addr = lane_addr + (slot ? C::S_COL1 : C::S_COL0);
+
+        // ---- S -> P: mask, running max with conditional O rescale, exponentials, row sum ----
+        uint32_t r[C::BN];
+#pragma unroll
+        for (int cc = 0; cc < C::BN / 32; ++cc) tmem_ld32(s_addr + cc * 32, r + cc * 32);
+        tmem_ld_wait();
+#pragma unroll
+        for (int cc = 0; cc < C::BN / 32; ++cc) tmem_reg_fence32(r + cc * 32);
+
+        const int kbase = j * C::BN;
+        // warp-uniform: does any key of this tile fall outside some row's visible range?
+        const bool need_mask =
+            (kbase + C::BN > args.Nkv) || (args.causal && kbase + C::BN - 1 > q_first + diag);
+        if (need_mask) {
+#pragma unroll
+          for (int i = 0; i < C::BN; ++i)
+            if (kbase + i > lim) r[i] = __float_as_uint(-INFINITY);
+        }
+        // row max: eight independent chains of 3-input max, then a short tree
+        float mx;
+        {
+          constexpr int Q8 = C::BN / 8;
+          float m8[8];
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            float a = __uint_as_float(r[kk * Q8]);
+#pragma unroll
+            for (int i = 1; i + 1 < Q8; i += 2)
+              a = fmax3(a, __uint_as_float(r[kk * Q8 + i]), __uint_as_float(r[kk * Q8 + i + 1]));
+            m8[kk] = (Q8 % 2 == 0) ? fmaxf(a, __uint_as_float(r[kk * Q8 + Q8 - 1])) : a;
+          }
+          mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+        }
+        const float m_new = fmaxf(m_ref, mx);
+        // true when the max moved by more than TAU (also on the first live tile: -inf -> finite)
+        const bool need = (m_new - m_ref) * c > kRescaleTau;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2((m_ref - m_new) * c) : 1.0f;
+          if (need) m_ref = m_new;
+          l *= alpha;
+          if (j > 0) {
+            if (C::NQT == 1) {
+              // PV of the previous tile must have landed in O before it is rescaled. (With two query
+              // tiles S_j is committed after PV_{j-1} of the same tile, so it has landed already.)
+              if (!wait_warp(o_done, uint32_t((t_run - 2) & 1))) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t o[32];
+              tmem_ld32(lane_addr + o_col + cc * 32, o);
+              tmem_ld_wait();
+              tmem_reg_fence32(o);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st32(lane_addr + o_col + cc * 32, o);
+            }
+            tmem_st_wait();
+          }
+        }
+        // P = 2^(c*s - c*m_ref) as bf16 over the first BN/2 columns of the slot (two per 32-bit
+        // column; the S values it replaces are already in registers). Pairs go through the packed
+        // FMA pipe; the exponential uses the exp unit (MUFU.EX2) or, for the last kEmuCols columns
+        // of tiles without masked keys, the FMA-pipe polynomial.
+        const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
+        const float2 c2 = make_float2(c, c);
+        const float2 nmc2 = make_float2(-mc, -mc);
+        float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                          make_float2(0.f, 0.f)};
+        constexpr int EMU_FROM = (C::BN - kEmuCols * C::BN / 128) / 2;  // first emulated pair
+        const bool emu = kEmuCols > 0 && !need_mask;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t p[C::HALF_PAIRS];
+#pragma unroll
+          for (int i2 = 0; i2 < C::HALF_PAIRS; ++i2) {
+            const int i = half * C::HALF_PAIRS + i2;
+            const float2 x =
+                ffma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nmc2);
+            float2 e;
+            if (i >= EMU_FROM && emu) {
+              e = exp2_poly2(x);
+            } else {
+              e.x = ex2(x.x);
+              e.y = ex2(x.y);
+            }
+            acc4[i & 3] = fadd2(acc4[i & 3], e);
+            p[i2] = pack_bf16x2(e.x, e.y);
+          }
+          if (C::HALF_PAIRS == 32)
+            tmem_st32(s_addr + half * C::HALF_PAIRS, p);
+          else
+            tmem_st16(s_addr + half * C::HALF_PAIRS, p);
+        }
+        warp_publish_tmem_stores(&p_full[slot], lane);
+        const float2 s01 = fadd2(acc4[0], acc4[1]);
+        const float2 s23 = fadd2(acc4[2], acc4[3]);
+        const float2 s = fadd2(s01, s23);
+        l += s.x + s.y;
+      }
+      if (!ok) break;
+
+      // ---- epilogue: O = acc / l (once), LSE = scale * m_ref + ln l -------------------------------
+      const bool valid = q_row < args.Nq;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.o) +
+                            ((size_t(un.b) * args.Nq + (valid ? q_row : 0)) * args.Hq + un.h) * D;
+      if (un.n_tiles > 0 && my_tiles == 0) {
+        // this tile saw no key, but the unit had MMAs: keep the o_final phase count in step
+        if (!wait_warp(&o_final[qt], uint32_t(uc & 1))) {
+          ok = false;
+          break;
+        }
+        ++uc;
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow);
+          for (int v4 = 0; v4 < D / 8; ++v4) dst[v4] = make_uint4(0, 0, 0, 0);
+        }
+      } else if (un.n_tiles > 0) {
+        if (!wait_warp(&o_final[qt], uint32_t(uc & 1))) {
+          ok = false;
+          break;
+        }
+        ++uc;
+        tc_fence_after();
+        const float inv = (l > 0.f) ? 1.0f / l : 0.f;
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
@@ -529,12 +641,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
           }
         }
+        // O of this tile was read (tcgen05.wait::ld above) before any P of the next unit is
+        // published, so the next unit's first PV cannot overwrite it early.
       } else if (valid) {
         uint4* dst = reinterpret_cast<uint4*>(orow);
         for (int v4 = 0; v4 < D / 8; ++v4) dst[v4] = make_uint4(0, 0, 0, 0);
       }
       if (valid)
-        args.lse[(size_t(b) * args.Hq + h) * args.Nq + q_row] =
+        args.lse[(size_t(un.b) * args.Hq + un.h) * args.Nq + q_row] =
             (l > 0.f) ? fmaf(m_ref, args.scale, logf(l)) : -INFINITY;
     }
   }
@@ -544,6 +658,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  // The last CTA to finish returns the scheduling slot to zero (all CTAs have stopped claiming).
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&g_sched_done[args.sched_slot], 1u) == gridDim.x - 1) {
+      atomicExch(&g_sched_next[args.sched_slot], 0u);
+      atomicExch(&g_sched_done[args.sched_slot], 0u);
+    }
   }
 }
 
@@ -593,7 +715,13 @@ static attn_status_t launch_fwd(const void* q, const void* k, const void* v, voi
   }
   const long long units = (long long)a.n_qblk * B * Hq;
   if (units > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
-  attn_fwd_kernel<D><<<dim3(unsigned(units)), dim3(C::THREADS), C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, a);
+  // persistent grid: one CTA per SM (each holds all 512 TMEM columns), walking the units in order
+  const int sms = sm_count();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  const unsigned grid = unsigned(units < sms ? units : sms);
+  static std::atomic<unsigned> launch_count{0};
+  a.sched_slot = int(launch_count.fetch_add(1) % kSchedSlots);
+  attn_fwd_kernel<D><<<dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, a);
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
 }
 

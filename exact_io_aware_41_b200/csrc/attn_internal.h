@@ -25,6 +25,7 @@ struct FwdArgs {
   int group;   // Hq / Hkv
   int n_qblk;  // query blocks of NQT*128 rows per (b, h)
   int heads_per_group;  // query heads per L2 group of units
+  int sched_slot;       // which unit-claim counter this launch uses
   int causal;
   float scale;       // natural-log scale on Q K^T
   float scale_log2;  // scale * log2(e)
@@ -34,6 +35,9 @@ struct FwdArgs {
 // A 4-d TMA map over a token-major bf16 tensor [outer, rows, heads, d] (d innermost), with a box
 // of `box_cols` elements of d x 1 head x `box_rows` tokens x 1 batch. Returns false on failure.
 bool is_aligned16(const void* p);
+
+// Streaming multiprocessors of the current device (-1 on error).
+int sm_count();
 
 bool encode_tile_map(CUtensorMap* map, const void* base, int d, int heads, int rows, int outer, int box_cols,
                      int box_rows, unsigned swizzle_bytes);
