@@ -44,8 +44,10 @@ struct DecCfg {
   static_assert(NV <= LPT, "one partial sum per lane group after the reduce-scatter");
 };
 
+// Eight query heads per kv head need 64 accumulator registers per lane: allow two CTAs per SM
+// (up to 255 registers) there, four CTAs (128 registers, 16 warps per SM) otherwise.
 template <int D, int G>
-__global__ void __launch_bounds__(kDecodeWarps * 32, 4)
+__global__ void __launch_bounds__(kDecodeWarps * 32, (G >= 8) ? 2 : 4)
     decode_split_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
                         const __nv_bfloat16* __restrict__ vc, const int32_t* __restrict__ kv_lens, int Nkv_cap,
                         int Hkv, int chunk, int n_splits, float scale_log2, float* __restrict__ part_o,
