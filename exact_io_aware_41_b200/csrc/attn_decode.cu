@@ -257,6 +257,246 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, (G >= 8) ? 2 : 4)
   }
 }
 
+// ============================================================================================
+// Split kernel, tensor-core variant (d = 64 or 128).
+//
+// A producer warp streams the CTA's K and V rows for its kv head through a STAGES-deep
+// shared-memory ring with TMA (tiles of TT tokens, 128-byte swizzle); the K/V rows are read from
+// HBM exactly once and never pass through registers on their way in. Each of the NW consumer warps
+// takes 16 tokens of every tile and does the two per-tile products on warp-level tensor cores
+// (mma.sync m16n8k16, bf16 in, fp32 accumulate): S = Q K^T with the group's query heads as the 16
+// rows (zero-padded past G), then O += P V with P taken straight from the S accumulators. The
+// online softmax runs on the accumulator fragments: lane (g, t) owns head g's scores for four of the
+// warp's tokens, so a row max is two shuffles. This keeps the per-token instruction count small
+// enough for the kernel to stay bound by HBM bandwidth.
+// ============================================================================================
+template <int D>
+struct DecTcCfg {
+  static constexpr int NW = 4;                  // consumer warps
+  static constexpr int TT = 16 * NW;            // tokens per tile
+  static constexpr int STAGES = 3;
+  static constexpr int NCHUNK = D / 64;         // 64-element (128-byte) swizzle chunks along d
+  static constexpr int CHUNK_BYTES = TT * 128;
+  static constexpr int TILE_BYTES = TT * D * 2;  // one K or V tile
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int THREADS = 32 * (NW + 1);
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 2 * STAGES * 8 + 16;
+};
+
+// Byte address of element (row, col) of a TT x D bf16 tile written by TMA with 128-byte swizzle:
+// 64-column chunks, 128-byte rows, the 16-byte unit index XOR-ed with the row index mod 8.
+template <int D>
+__device__ __forceinline__ uint32_t dec_sw128(uint32_t tile, int row, int col) {
+  const int chunk = col >> 6, unit = (col & 63) >> 3;
+  return tile + chunk * DecTcCfg<D>::CHUNK_BYTES + row * 128 + ((unit ^ (row & 7)) << 4) + ((col & 7) << 1);
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(DecTcCfg<D>::THREADS, 2)
+    decode_split_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                           const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ kv_lens, int Nkv_cap,
+                           int Hkv, int chunk, int n_splits, float scale_log2, float* __restrict__ part_o,
+                           float* __restrict__ part_lse, unsigned long long timeout_ns) {
+  using C = DecTcCfg<D>;
+  static_assert(G <= 8, "query heads of a group fill at most the upper half of the 16 MMA rows");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + C::STAGES);
+  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Hq = Hkv * G;
+  const uint64_t T = timeout_ns;
+
+  int L = kv_lens[b];
+  if (L < 0 || L > Nkv_cap) {
+    if (threadIdx.x == 0 && s == 0 && g == 0) atomicOr(&g_error_word, kErrBadLengthBit);
+    L = L < 0 ? 0 : Nkv_cap;
+  }
+  const int t_begin = s * chunk;
+  const int t_end = min(L, t_begin + chunk);
+  const size_t row0 = size_t(b) * Hq + size_t(g) * G;  // first query head row of this group
+  if (t_begin >= t_end) {
+    if (threadIdx.x < G) part_lse[(row0 + threadIdx.x) * n_splits + s] = -INFINITY;
+    return;
+  }
+  const int n_tiles = (t_end - t_begin + C::TT - 1) / C::TT;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], C::NW);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == C::NW) {
+    // ================================ TMA producer ================================
+    if (lane == 0) {
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      int i = 0;
+      for (; i < n_tiles; ++i) {
+        const int st = i % C::STAGES;
+        if (!mbar_wait(&empty[st], uint32_t(((i / C::STAGES) & 1) ^ 1), abort_flag, T)) break;
+        mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
+        uint8_t* kt = smem + st * C::STAGE_BYTES;
+        const int tok = t_begin + i * C::TT;
+#pragma unroll
+        for (int c = 0; c < C::NCHUNK; ++c) {
+          tma_load_4d(kt + c * C::CHUNK_BYTES, &tmK, &full[st], c * 64, g, tok, b);
+          tma_load_4d(kt + C::TILE_BYTES + c * C::CHUNK_BYTES, &tmV, &full[st], c * 64, g, tok, b);
+        }
+      }
+      if (i < n_tiles) {
+        // gave up: let the copies in flight land before the CTA exits
+        for (int st = 0; st < C::STAGES; ++st) {
+          const int fills = (i - st + C::STAGES - 1) / C::STAGES;
+          if (fills > 0) mbar_wait(&full[st], (fills - 1) & 1, nullptr, 100000000ull);
+        }
+      }
+    }
+    return;  // the consumers' closing barrier below counts only the consumer warps
+  }
+
+  // ================================ consumer warps ================================
+  const int gid = lane >> 2, tid = lane & 3;  // mma fragment coordinates
+  // A fragments of Q (rows = query heads of the group, zero past G), one pair per 16-wide k-step
+  uint32_t qa[D / 16][2];
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    if (gid < G) {
+      const __nv_bfloat16* qr = q + (row0 + gid) * D + kk * 16 + 2 * tid;
+      qa[kk][0] = *reinterpret_cast<const uint32_t*>(qr);
+      qa[kk][1] = *reinterpret_cast<const uint32_t*>(qr + 8);
+    } else {
+      qa[kk][0] = qa[kk][1] = 0u;
+    }
+  }
+  float o[D / 8][4];  // O rows gid (and padding rows gid + 8), columns 8n + 2t, 8n + 2t + 1
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m_ref = -INFINITY;  // head gid's reference max (log2 units of the scaled scores)
+  float l = 0.f;            // partial sum of p over this lane's tokens
+  const int mi = lane >> 3, rr = lane & 7;  // ldmatrix: which 8x8 matrix this lane addresses, and its row
+
+  bool ok = true;
+  for (int i = 0; i < n_tiles; ++i) {
+    const int st = i % C::STAGES;
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[st], uint32_t((i / C::STAGES) & 1), abort_flag, T))) {
+      ok = false;
+      break;
+    }
+    const uint32_t kt = smem_u32(smem + st * C::STAGE_BYTES);
+    const uint32_t vt = kt + C::TILE_BYTES;
+    const int my_tok0 = t_begin + i * C::TT + 16 * warp;  // this warp's tokens: my_tok0 .. my_tok0 + 15
+    const int valid = t_end - my_tok0;                     // how many of them exist
+    if (valid > 0) {
+      // ---- S = Q K^T over 16 tokens (two 8-token column blocks)
+      float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t b00, b01, b10, b11;
+        ldsm_x4(dec_sw128<D>(kt, 16 * warp + 8 * (mi >> 1) + rr, kk * 16 + 8 * (mi & 1)), b00, b01, b10, b11);
+        mma_bf16_16816(sacc[0], qa[kk][0], 0u, qa[kk][1], 0u, b00, b01);
+        mma_bf16_16816(sacc[1], qa[kk][0], 0u, qa[kk][1], 0u, b10, b11);
+      }
+      // scores of head gid for tokens 2t, 2t+1, 8+2t, 9+2t (log2 units); tokens past t_end are -inf
+      float x[4] = {sacc[0][0] * scale_log2, sacc[0][1] * scale_log2, sacc[1][0] * scale_log2,
+                    sacc[1][1] * scale_log2};
+      const int tk[4] = {2 * tid, 2 * tid + 1, 8 + 2 * tid, 9 + 2 * tid};
+      float mx = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (tk[k] >= valid) x[k] = -INFINITY;
+        mx = fmaxf(mx, x[k]);
+      }
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));  // max over the warp's 16 tokens
+      if (mx - m_ref > kDecodeTau) {                          // conditional rescale (first tile: always)
+        const float alpha = ex2(m_ref - mx);
+        l *= alpha;
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+          o[n][0] *= alpha;
+          o[n][1] *= alpha;
+        }
+        m_ref = mx;
+      }
+      float pv[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        pv[k] = (x[k] == -INFINITY) ? 0.f : ex2(x[k] - m_ref);
+        l += pv[k];
+      }
+      const uint32_t pa0 = pack_bf16x2(pv[0], pv[1]);  // P[gid][tokens 2t, 2t+1]
+      const uint32_t pa2 = pack_bf16x2(pv[2], pv[3]);  // P[gid][tokens 8+2t, 9+2t]
+      // V rows past the end of the sequence may hold anything (0 * NaN would poison O): zero them
+      if (valid < 16) {
+        const int first = valid < 0 ? 0 : valid;
+        for (int idx = lane; idx < (16 - first) * (D / 8); idx += 32) {
+          const int r = first + idx / (D / 8), unit = idx % (D / 8);
+          const uint32_t a = vt + (unit >> 3) * C::CHUNK_BYTES + (16 * warp + r) * 128 + ((unit & 7) << 4);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
+        }
+        __syncwarp();
+      }
+      // ---- O += P V (16-column blocks of d: one transposed ldmatrix, two MMAs)
+#pragma unroll
+      for (int db = 0; db < D / 16; ++db) {
+        uint32_t v00, v01, v10, v11;
+        ldsm_x4_t(dec_sw128<D>(vt, 16 * warp + 8 * (mi & 1) + rr, 16 * db + 8 * (mi >> 1)), v00, v01, v10, v11);
+        mma_bf16_16816(o[2 * db], pa0, 0u, pa2, 0u, v00, v01);
+        mma_bf16_16816(o[2 * db + 1], pa0, 0u, pa2, 0u, v10, v11);
+      }
+      if (valid < 16) fence_proxy_async_smem();  // the zeroing writes precede the next TMA into the stage
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+  }
+
+  // ---- merge the consumer warps (the ring is idle now: every tile has been consumed)
+  l += __shfl_xor_sync(0xffffffffu, l, 1);
+  l += __shfl_xor_sync(0xffffffffu, l, 2);
+  float* sm_m = reinterpret_cast<float*>(smem);   // [NW][G]
+  float* sm_l = sm_m + C::NW * G;                 // [NW][G]
+  float* sm_acc = sm_l + C::NW * G;               // [NW][G][D]
+  asm volatile("bar.sync 1, %0;" ::"n"(C::NW * 32) : "memory");  // all consumers are done with the ring
+  if (gid < G) {
+    if (tid == 0) {
+      sm_m[warp * G + gid] = ok ? m_ref : -INFINITY;
+      sm_l[warp * G + gid] = l;
+    }
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      sm_acc[(warp * G + gid) * D + 8 * n + 2 * tid] = o[n][0];
+      sm_acc[(warp * G + gid) * D + 8 * n + 2 * tid + 1] = o[n][1];
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(C::NW * 32) : "memory");
+  for (int idx = threadIdx.x; idx < G * D; idx += C::NW * 32) {
+    const int hh = idx / D, e = idx % D;
+    float m = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < C::NW; ++w) m = fmaxf(m, sm_m[w * G + hh]);
+    float lt = 0.f, ot = 0.f;
+    if (m != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < C::NW; ++w) {
+        const float f = ex2(sm_m[w * G + hh] - m);
+        lt = fmaf(f, sm_l[w * G + hh], lt);
+        ot = fmaf(f, sm_acc[(w * G + hh) * D + e], ot);
+      }
+    }
+    const size_t row = row0 + hh;
+    part_o[(row * n_splits + s) * D + e] = (lt > 0.f) ? ot / lt : 0.f;
+    if (e == 0) part_lse[row * n_splits + s] = (lt > 0.f) ? (m * 0.6931471805599453f + logf(lt)) : -INFINITY;
+  }
+}
+
 // One CTA per output row; each thread owns EPT consecutive elements of d. The partial LSEs are
 // reduced first, the live splits are compacted into a list in shared memory, and the partial
 // outputs are accumulated with four independent loads in flight per thread.
@@ -358,12 +598,12 @@ __global__ void __launch_bounds__(CombCfg<D>::NT)
 // host side
 // ---------------------------------------------------------------------------------------------
 int decode_default_chunk(int B, int Hkv, int Nkv_cap) {
-  // aim for ~8 live CTAs per SM if every sequence were full, in multiples of 64 tokens, at most 1024
+  // aim for ~8 live CTAs per SM if every sequence were full, in multiples of 64 tokens, at most 2048
   const long long total = (long long)B * Hkv * Nkv_cap;
   long long c = total / (148LL * 8);
   c = (c + 63) / 64 * 64;
   if (c < 64) c = 64;
-  if (c > 1024) c = 1024;
+  if (c > 2048) c = 2048;
   return int(c);
 }
 
@@ -386,16 +626,51 @@ static attn_status_t launch_split(const void* q, const void* kc, const void* vc,
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
 }
 
+template <int D, int G>
+static attn_status_t launch_split_tc(const void* q, const void* kc, const void* vc, const int32_t* lens, int cap,
+                                     int B, int Hkv, int chunk, int n_splits, float scale, float* po, float* pl,
+                                     cudaStream_t stream) {
+  using C = DecTcCfg<D>;
+  CUtensorMap tmK, tmV;
+  if (!encode_tile_map(&tmK, kc, D, Hkv, cap, B, 64, C::TT, 128) ||
+      !encode_tile_map(&tmV, vc, D, Hkv, cap, B, 64, C::TT, 128))
+    return ATTN_ERR_CUDA;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(decode_split_tc_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_BYTES) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    attr_set = true;
+  }
+  dim3 grid(n_splits, Hkv, B);
+  decode_split_tc_kernel<D, G><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(
+      tmK, tmV, reinterpret_cast<const __nv_bfloat16*>(q), lens, cap, Hkv, chunk, n_splits,
+      scale * 1.4426950408889634f, po, pl, kWaitLimitNs);
+  return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
+}
+
+// d = 64 and 128 use the tensor-core split kernel; d = 256 (whose O fragments would not fit the
+// register budget) uses the CUDA-core one.
 template <int D>
 static attn_status_t split_by_group(int G, const void* q, const void* kc, const void* vc, const int32_t* lens,
                                     int cap, int B, int Hkv, int chunk, int n_splits, float scale, float* po,
                                     float* pl, cudaStream_t st) {
-  switch (G) {
-    case 1: return launch_split<D, 1>(q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
-    case 2: return launch_split<D, 2>(q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
-    case 4: return launch_split<D, 4>(q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
-    case 8: return launch_split<D, 8>(q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
-    default: return ATTN_ERR_UNSUPPORTED;
+  if constexpr (D <= 128) {
+    switch (G) {
+      case 1: return launch_split_tc<D, 1>(q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
+      case 2: return launch_split_tc<D, 2>(q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
+      case 4: return launch_split_tc<D, 4>(q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
+      case 8: return launch_split_tc<D, 8>(q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
+      default: return ATTN_ERR_UNSUPPORTED;
+    }
+  } else {
+    switch (G) {
+      case 1: return launch_split<D, 1>(q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
+      case 2: return launch_split<D, 2>(q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
+      case 4: return launch_split<D, 4>(q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
+      case 8: return launch_split<D, 8>(q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
+      default: return ATTN_ERR_UNSUPPORTED;
+    }
   }
 }
 
