@@ -101,6 +101,11 @@ class ClockSampler:
 # distributed plumbing
 # ------------------------------------------------------------------------------------------------
 def dist_setup(n_gpus: int):
+    """Rank, world and the process group from the torchrun environment (NCCL on GPUs, gloo on CPUs).
+
+    The group carries only the barrier around the timed region and the max-over-ranks reduction of
+    the timings: every rank runs an independent problem, nothing on the data path is exchanged.
+    """
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -110,12 +115,24 @@ def dist_setup(n_gpus: int):
     if world > 1:
         import datetime
 
+        import torch
         import torch.distributed as dist
 
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=None)
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
         pg = dist
     return world, rank, local, pg
+
+
+def max_over_ranks(values, dist, device=None):
+    """Element-wise maximum of a list of floats over all ranks (the slowest rank's times)."""
+    if dist is None:
+        return list(values)
+    import torch
+
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
 
 
 def physical_gpu(local: int) -> int:
@@ -260,10 +277,7 @@ def run_ours(args, world, rank, local, dist):
     total_ms = t_start.elapsed_time(t_end)
     pf_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
     dec_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
-    times = torch.tensor([total_ms, pf_ms, dec_ms], dtype=torch.float64, device=dev)
-    if dist:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-    total_ms, pf_ms, dec_ms = times.tolist()
+    total_ms, pf_ms, dec_ms = max_over_ranks([total_ms, pf_ms, dec_ms], dist, dev)
     err = lib.attn_get_last_error()
     if err != lib.ATTN_OK:
         raise SystemExit(f"device error word after the timed region: {lib.status_string(err)}")
@@ -288,12 +302,9 @@ def run_ours(args, world, rank, local, dist):
     # ---- end to end through the public API with pinned host buffers
     e2e = e2e_prefill(lib, P, q, k, v, stream, max(3, min(K, 50)))
     dec_e2e = e2e_decode(lib, Dw, dq, kc, vc, lens_np, stream, 2) if not args.no_e2e_decode else None
-    if dist:
-        t = torch.tensor([e2e["ms"], (dec_e2e or {}).get("ms", 0.0)], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e["ms"], dms = t.tolist()
-        if dec_e2e:
-            dec_e2e["ms"] = dms
+    e2e["ms"], dms = max_over_ranks([e2e["ms"], (dec_e2e or {}).get("ms", 0.0)], dist, dev)
+    if dec_e2e:
+        dec_e2e["ms"] = dms
 
     if rank != 0:
         return None
@@ -335,7 +346,7 @@ def run_ours(args, world, rank, local, dist):
             "value": dec_value, "unit": "GB/s", "ms_per_call": dec_avg_s * 1e3,
             "algorithmic_bytes_per_call": dec_bytes,
             "frac_of_nominal_hbm": dec_gbs_1 / NOMINAL_HBM_GBS,
-            "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<128,4> + decode_combine_kernel<128>",
+            "roofline": {"bound": "hbm", "kernel": "decode_split_tc_kernel<128,4> + decode_combine_kernel<128>",
                          "achieved": dec_gbs_1, "peak": meas_bw, "unit": "GB/s", "frac": dec_gbs_1 / meas_bw,
                          "peak_source": f"{peak_src} copy bandwidth", "traffic": args.decode_traffic},
             "e2e": dec_e2e and {

@@ -146,7 +146,7 @@ attn_status_t attn_get_last_error(void);
 const char* attn_status_string(attn_status_t status);
 
 /*
- * Name of the kernel that `which` selects (0 = prefill forward, 1 = decode split, 2 = decode
+ * Name of the kernel(s) that `which` selects (0 = prefill forward, 1 = decode split, 2 = decode
  * combine), for recording which kernel a measurement ran (the evolution article's section 1.1
  * asks that a benchmark name its kernel). Returns NULL for an unknown index.
  */
