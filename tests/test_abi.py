@@ -54,7 +54,7 @@ def test_status_strings_and_kernel_names():
     assert "timed out" in pkg.status_string(pkg.ATTN_ERR_TIMEOUT)
     assert pkg.status_string(99) == "unknown status"
     assert pkg.kernel_name(0).startswith("attn::attn_fwd_kernel")
-    assert pkg.kernel_name(1).startswith("attn::decode_split_kernel")
+    assert pkg.kernel_name(1).startswith("attn::decode_split_tc_kernel")
     assert pkg.kernel_name(7) is None
 
 
