@@ -21,8 +21,11 @@
 // core: while one tile's softmax runs, the other tile's MMAs run ("overlaps multiple query tiles",
 // section 5). With d = 256 one query tile alternates between two S buffers instead.
 //
-// S and P never leave the SM: S is fp32 in TMEM, P is bf16 written in place over S and read by
-// the MMA straight from TMEM.
+// S and P never leave the SM: S is fp32 in TMEM, P is bf16 in TMEM, read by the MMA straight from
+// there. At d = 128 (and 256) P is written in place over S, so a tile's next S = Q K^T waits for
+// the PV that reads P. At d <= 64 the O accumulators are narrow enough to leave TMEM columns for
+// P buffers of its own: the next S of a tile is computed as soon as the softmax has read the
+// current one, overlapping that tile's own softmax.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -73,6 +76,10 @@ struct FwdCfg {
   static constexpr int BM = 128;                        // query rows per tile (TMEM lanes)
   static constexpr int NQT = (D <= 128) ? 2 : 1;        // query tiles per CTA
   static constexpr int BN = (D <= 128) ? 128 : 64;      // keys per K/V tile
+  // d <= 64: P lives in tensor-memory buffers of its own instead of over S, so a tile's next
+  // S = Q K^T is computed while the softmax still works on the current one (the two O accumulators
+  // leave room for the buffers). d = 128 has no room for them and writes P over S.
+  static constexpr bool SEP_P = (NQT == 2) && (D < 128);
   static constexpr int CHUNK = (D >= 64) ? 64 : 32;     // elements per swizzled smem row
   static constexpr int NCHUNK = D / CHUNK;              // swizzle chunks along d
   static constexpr int ROWB = CHUNK * 2;                // bytes per swizzled row (128 or 64)
@@ -82,7 +89,7 @@ struct FwdCfg {
   static constexpr int KV_CHUNK_BYTES = BN * ROWB;
   static constexpr int Q_TILE_BYTES = BM * D * 2;
   static constexpr int KV_TILE_BYTES = BN * D * 2;
-  static constexpr int STAGES = (D == 128 || D == 256) ? 4 : 8;
+  static constexpr int STAGES = (KV_TILE_BYTES >= 32768) ? 4 : 8;
   static constexpr int NSMWG = (NQT == 2) ? 2 : 1;      // softmax warpgroups
   static constexpr int THREADS = 128 * (1 + NSMWG);
   static constexpr int HALF_PAIRS = BN / 4;             // bf16 pairs (TMEM columns) of P per half tile
@@ -92,12 +99,15 @@ struct FwdCfg {
   static constexpr int S_COL1 = BN;
   static constexpr int O_COL0 = 2 * BN;
   static constexpr int O_COL1 = 2 * BN + D;
+  // separate P buffers (bf16 pairs: BN / 2 columns each), after the O accumulators
+  static constexpr int P_COL0 = 2 * BN + NQT * D;
+  static constexpr int P_COL1 = P_COL0 + BN / 2;
   static constexpr int TMEM_COLS = 512;
-  static_assert(2 * BN + NQT * D <= TMEM_COLS, "tensor memory budget");
+  static_assert(2 * BN + NQT * D + (SEP_P ? NQT * BN / 2 : 0) <= TMEM_COLS, "tensor memory budget");
   // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done, o_final[2], drain,
-  // sched_full[SCHED], sched_empty[SCHED]
+  // s_free[2], p_free[2], sched_full[SCHED], sched_empty[SCHED]
   static constexpr int SCHED = 4;  // units the producer may claim ahead of the consumers
-  static constexpr int NBARS = 2 + 2 * STAGES + 2 + 2 + 1 + 2 + 1 + 2 * SCHED;
+  static constexpr int NBARS = 2 + 2 * STAGES + 2 + 2 + 1 + 2 + 1 + 2 + 2 + 2 * SCHED;
   static constexpr int SCHED_CONSUMERS = 1 + 4 * NSMWG;  // MMA thread + one arrival per softmax warp
   static constexpr int SMEM_DATA = NQT * Q_TILE_BYTES + STAGES * KV_TILE_BYTES;
   // Pad small-d configurations so only one CTA (and one 512-column TMEM allocation) fits per SM.
@@ -179,7 +189,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   uint64_t* o_done = p_full + 2;            // one phase per PV (single-tile path: O rescale needs PV_{j-1})
   uint64_t* o_final = o_done + 1;           // [tile] one phase per unit: every MMA of the unit is done
   uint64_t* drain = o_final + 2;            // error path: MMAs in flight have finished
-  uint64_t* sched_full = drain + 1;         // [SCHED] the producer wrote the k-th unit index
+  uint64_t* s_free = drain + 1;             // [tile] separate P: the softmax has read S (one phase per S)
+  uint64_t* p_free = s_free + 2;            // [tile] separate P: the PV reading the P buffer is done
+  uint64_t* sched_full = p_free + 2;        // [SCHED] the producer wrote the k-th unit index
   uint64_t* sched_empty = sched_full + C::SCHED;  // [SCHED] every role read it
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sched_empty + C::SCHED);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -203,6 +215,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4);  // one arrival per softmax warp
       mbar_init(&o_final[i], 1);
+      mbar_init(&s_free[i], 4);  // one arrival per softmax warp of the tile
+      mbar_init(&p_free[i], 1);
     }
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
@@ -353,6 +367,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       int pos = 0;    // ring position of the next K/V tile to consume
       int qc = 0;     // units issued (phase of q_full)
       int pc[2] = {0, 0};  // P tiles consumed per slot (phase of p_full)
+      int qk_cnt[2] = {0, 0};  // separate P: S tiles issued per query tile (phase of s_free)
       int t_run = 0;  // single-tile path: S tiles issued so far (slot = t_run & 1)
       for (int k = 0; ok; ++k) {
         const int lin = next_unit(k, false);
@@ -363,7 +378,50 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         ok = mbar_wait(q_full, qc & 1, abort_flag, T);
         ++qc;
         const int base = pos;  // K_j at base + 2j, V_j at base + 2j + 1
-        if (C::NQT == 2) {
+        if (C::SEP_P) {
+          // Two query tiles, P in buffers of its own. QK(t, j+1) may overwrite S once the softmax has
+          // read S(t, j) (s_free); PV(t, j) reads P(t, j) once it is in place (p_full) and frees the
+          // buffer when done (p_free):  QK(0,0) QK(1,0) | QK(0,1) QK(1,1) PV(0,0) PV(1,0) | ...
+          const int nt[2] = {un.n_tile0, n};
+          auto qk_into = [&](int qt, int stage) -> bool {
+            if (qk_cnt[qt] > 0) {
+              if (!mbar_wait(&s_free[qt], uint32_t((qk_cnt[qt] - 1) & 1), abort_flag, T)) return false;
+              tc_fence_after();
+            }
+            issue_qk(qt, qt ? C::S_COL1 : C::S_COL0, stage);
+            umma_commit(&s_full[qt]);
+            ++qk_cnt[qt];
+            return true;
+          };
+          if (ok) ok = mbar_wait(&kv_full[kv_slot(base)], kv_phase(base), abort_flag, T);
+#pragma unroll
+          for (int qt = 0; qt < 2; ++qt)
+            if (ok && nt[qt] > 0) ok = qk_into(qt, kv_slot(base));
+          if (ok) umma_commit(&kv_empty[kv_slot(base)]);
+          for (int j = 0; j < n && ok; ++j) {
+            const int pv_pos = base + 2 * j + 1, pk_pos = base + 2 * j + 2;
+            const bool nxt = j + 1 < n;
+            ok = mbar_wait(&kv_full[kv_slot(pv_pos)], kv_phase(pv_pos), abort_flag, T);
+            if (ok && nxt) ok = mbar_wait(&kv_full[kv_slot(pk_pos)], kv_phase(pk_pos), abort_flag, T);
+#pragma unroll
+            for (int qt = 0; qt < 2; ++qt)
+              if (ok && j + 1 < nt[qt]) ok = qk_into(qt, kv_slot(pk_pos));
+#pragma unroll
+            for (int qt = 0; qt < 2; ++qt) {
+              if (!ok || j >= nt[qt]) continue;
+              ok = mbar_wait(&p_full[qt], pc[qt] & 1, abort_flag, T);
+              if (!ok) break;
+              ++pc[qt];
+              tc_fence_after();
+              issue_pv(qt ? C::O_COL1 : C::O_COL0, qt ? C::P_COL1 : C::P_COL0, kv_slot(pv_pos), j > 0);
+              umma_commit(&p_free[qt]);
+            }
+            if (!ok) break;
+            umma_commit(&kv_empty[kv_slot(pv_pos)]);
+            if (nxt) umma_commit(&kv_empty[kv_slot(pk_pos)]);
+          }
+          pos = base + 2 * n;
+        } else if (C::NQT == 2) {
           // Two query tiles, one S slot each: QK(0,0) QK(1,0) | PV(0,j) QK(0,j+1) PV(1,j) QK(1,j+1) | ...
           if (ok) ok = mbar_wait(&kv_full[kv_slot(base)], kv_phase(base), abort_flag, T);
           // a causal unit's first query tile may need one K/V tile fewer than the second
@@ -472,6 +530,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     int sc = 0;     // S tiles consumed by this warpgroup (two tiles: phase of s_full[qt])
     int t_run = 0;  // single-tile path: S tiles consumed so far (slot = t_run & 1)
     int uc = 0;     // units with keys finished (phase of o_final)
+    int pt = 0;     // separate P: P tiles this warpgroup has published (phase of p_free[qt])
     for (int k = 0; ok; ++k) {
       const int lin = next_unit(k, true);
       if (lin < 0) break;
@@ -496,6 +555,15 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         ++t_run;
         tc_fence_after();
         const uint32_t s_addr = lane_addr + (slot ? C::S_COL1 : C::S_COL0);
+        // where P goes: a buffer of its own, or over S
+        const uint32_t p_addr = C::SEP_P ? lane_addr + (slot ? C::P_COL1 : C::P_COL0) : s_addr;
+        // separate P: the previous PV of this tile (it reads the P buffer and adds into O) is done
+        auto wait_prev_pv = [&]() -> bool {
+          if (!C::SEP_P || pt == 0) return true;
+          if (!wait_warp(&p_free[slot], uint32_t((pt - 1) & 1))) return false;
+          tc_fence_after();
+          return true;
+        };
 
         // ---- S -> P: mask, running max with conditional O rescale, exponentials, row sum ----
         uint32_t r[C::BN];
@@ -504,6 +572,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         tmem_ld_wait();
 #pragma unroll
         for (int cc = 0; cc < C::BN / 32; ++cc) tmem_reg_fence32(r + cc * 32);
+        if (C::SEP_P) {
+          // S is in registers: the next QK of this tile may overwrite it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_free[slot]);
+        }
 
         const int kbase = j * C::BN;
         // warp-uniform: does any key of this tile fall outside some row's visible range?
@@ -539,12 +613,16 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           if (j > 0) {
             if (C::NQT == 1) {
               // PV of the previous tile must have landed in O before it is rescaled. (With two query
-              // tiles S_j is committed after PV_{j-1} of the same tile, so it has landed already.)
+              // tiles and P over S, S_j is committed after PV_{j-1} of the same tile, so it has
+              // landed already; with separate P it is waited for here.)
               if (!wait_warp(o_done, uint32_t((t_run - 2) & 1))) {
                 ok = false;
                 break;
               }
               tc_fence_after();
+            } else if (!wait_prev_pv()) {
+              ok = false;
+              break;
             }
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {
@@ -570,6 +648,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                           make_float2(0.f, 0.f)};
         constexpr int EMU_FROM = (C::BN - kEmuCols * C::BN / 128) / 2;  // first emulated pair
         const bool emu = kEmuCols > 0 && !need_mask;
+        if (!wait_prev_pv()) {  // the P buffer is free again
+          ok = false;
+          break;
+        }
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t p[C::HALF_PAIRS];
@@ -589,11 +671,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             p[i2] = pack_bf16x2(e.x, e.y);
           }
           if (C::HALF_PAIRS == 32)
-            tmem_st32(s_addr + half * C::HALF_PAIRS, p);
+            tmem_st32(p_addr + half * C::HALF_PAIRS, p);
           else
-            tmem_st16(s_addr + half * C::HALF_PAIRS, p);
+            tmem_st16(p_addr + half * C::HALF_PAIRS, p);
         }
         warp_publish_tmem_stores(&p_full[slot], lane);
+        ++pt;
         const float2 s01 = fadd2(acc4[0], acc4[1]);
         const float2 s23 = fadd2(acc4[2], acc4[3]);
         const float2 s = fadd2(s01, s23);
