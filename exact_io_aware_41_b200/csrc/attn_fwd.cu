@@ -315,7 +315,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         const Unit un = unit_at<D>(args, lin);
         if (un.n_tiles == 0) continue;
         const int g = un.h / args.group;
-        // Q of the previous unit must be consumed by all its MMAs before it is overwritten
+        // Q of the previous unit must be consumed by all its QK MMAs before it is overwritten
         if (qc > 0 && !mbar_wait(q_empty, (qc - 1) & 1, abort_flag, T)) {
           ok = false;
           break;
@@ -383,20 +383,21 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           // read S(t, j) (s_free); PV(t, j) reads P(t, j) once it is in place (p_full) and frees the
           // buffer when done (p_free):  QK(0,0) QK(1,0) | QK(0,1) QK(1,1) PV(0,0) PV(1,0) | ...
           const int nt[2] = {un.n_tile0, n};
-          auto qk_into = [&](int qt, int stage) -> bool {
+          auto qk_into = [&](int qt, int jj, int stage) -> bool {
             if (qk_cnt[qt] > 0) {
               if (!mbar_wait(&s_free[qt], uint32_t((qk_cnt[qt] - 1) & 1), abort_flag, T)) return false;
               tc_fence_after();
             }
             issue_qk(qt, qt ? C::S_COL1 : C::S_COL0, stage);
             umma_commit(&s_full[qt]);
+            if (qt == 1 && jj == n - 1) umma_commit(q_empty);  // the unit's last QK: Q may be reloaded
             ++qk_cnt[qt];
             return true;
           };
           if (ok) ok = mbar_wait(&kv_full[kv_slot(base)], kv_phase(base), abort_flag, T);
 #pragma unroll
           for (int qt = 0; qt < 2; ++qt)
-            if (ok && nt[qt] > 0) ok = qk_into(qt, kv_slot(base));
+            if (ok && nt[qt] > 0) ok = qk_into(qt, 0, kv_slot(base));
           if (ok) umma_commit(&kv_empty[kv_slot(base)]);
           for (int j = 0; j < n && ok; ++j) {
             const int pv_pos = base + 2 * j + 1, pk_pos = base + 2 * j + 2;
@@ -405,7 +406,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             if (ok && nxt) ok = mbar_wait(&kv_full[kv_slot(pk_pos)], kv_phase(pk_pos), abort_flag, T);
 #pragma unroll
             for (int qt = 0; qt < 2; ++qt)
-              if (ok && j + 1 < nt[qt]) ok = qk_into(qt, kv_slot(pk_pos));
+              if (ok && j + 1 < nt[qt]) ok = qk_into(qt, j + 1, kv_slot(pk_pos));
 #pragma unroll
             for (int qt = 0; qt < 2; ++qt) {
               if (!ok || j >= nt[qt]) continue;
@@ -432,6 +433,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               if (nt[qt] == 0) continue;
               issue_qk(qt, qt ? C::S_COL1 : C::S_COL0, kv_slot(base));
               umma_commit(&s_full[qt]);
+              if (qt == 1 && n == 1) umma_commit(q_empty);  // the unit's last QK: Q may be reloaded
             }
             umma_commit(&kv_empty[kv_slot(base)]);
           }
@@ -455,6 +457,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               if (j + 1 < nt[qt]) {
                 issue_qk(qt, s_col, kv_slot(pk_pos));
                 umma_commit(&s_full[qt]);
+                if (qt == 1 && j + 2 == n) umma_commit(q_empty);  // the unit's last QK
               }
             }
             if (!ok) break;
@@ -470,6 +473,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             if (!ok) break;
             issue_qk(0, ((t0 + j) & 1) ? C::S_COL1 : C::S_COL0, kv_slot(base + 2 * j));
             umma_commit(&s_full[(t0 + j) & 1]);
+            if (j == n - 1) umma_commit(q_empty);  // the unit's last QK: Q may be reloaded
             umma_commit(&kv_empty[kv_slot(base + 2 * j)]);
           }
           for (int j = 0; j < n && ok; ++j) {
@@ -489,6 +493,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               if (!ok) break;
               issue_qk(0, s_col, kv_slot(kp));
               umma_commit(&s_full[slot]);
+              if (j + 3 == n) umma_commit(q_empty);  // the unit's last QK
               umma_commit(&kv_empty[kv_slot(kp)]);
             }
           }
@@ -496,8 +501,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           pos = base + 2 * n;
         }
         if (!ok) break;
-        // every MMA of this unit done: Q may be reloaded, O may be read (one o_final per tile)
-        umma_commit(q_empty);
+        // every MMA of this unit done: O may be read (one o_final per tile). (Q was released after the
+        // unit's last QK, so the next unit's Q load overlaps the last PVs and the epilogue.)
         umma_commit(&o_final[0]);
         if (C::NQT == 2) umma_commit(&o_final[1]);
       }

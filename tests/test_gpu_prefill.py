@@ -67,6 +67,15 @@ def test_large_score_spread(lib):
     _run_small(lib, 4102, 1, 2, 2, 384, 384, 256, True, scale=1.5)
 
 
+@pytest.mark.parametrize("d", [32, 64])
+def test_small_head_dims_rescale_and_units_per_cta(lib, d):
+    # d <= 64 keeps P in buffers of its own; a large scale makes the running max jump (O rescales that
+    # must wait for the previous PV), and 384 causal units on the persistent grid give every CTA
+    # several units, so the S and P hand-off counters carry across units
+    _run_small(lib, 4300 + d, 1, 2, 2, 512, 512, d, False, scale=1.5)
+    _run_small(lib, 4310 + d, 4, 16, 4, 1300, 1300, d, True, scale=0.6)
+
+
 def test_repeat_calls_are_identical(lib):
     import torch
 
