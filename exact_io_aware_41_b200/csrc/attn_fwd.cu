@@ -89,7 +89,7 @@ struct FwdCfg {
   static constexpr int KV_CHUNK_BYTES = BN * ROWB;
   static constexpr int Q_TILE_BYTES = BM * D * 2;
   static constexpr int KV_TILE_BYTES = BN * D * 2;
-  static constexpr int STAGES = (KV_TILE_BYTES >= 32768) ? 4 : 8;
+  static constexpr int STAGES = (D == 256) ? 5 : (KV_TILE_BYTES >= 32768) ? 4 : 8;
   static constexpr int NSMWG = (NQT == 2) ? 2 : 1;      // softmax warpgroups
   static constexpr int THREADS = 128 * (1 + NSMWG);
   static constexpr int HALF_PAIRS = BN / 4;             // bf16 pairs (TMEM columns) of P per half tile
@@ -102,8 +102,14 @@ struct FwdCfg {
   // separate P buffers (bf16 pairs: BN / 2 columns each), after the O accumulators
   static constexpr int P_COL0 = 2 * BN + NQT * D;
   static constexpr int P_COL1 = P_COL0 + BN / 2;
+  // d = 256: the Q tile is copied into TMEM (bf16 pairs, D / 2 columns) once per unit and QK reads
+  // it from there, so the 64-key QK MMAs read only K from shared memory (with Q from shared memory
+  // as well they are shared-memory bound at N = 64)
+  static constexpr bool Q_TMEM = (D == 256);
+  static constexpr int Q_COL = 2 * BN + NQT * D;
   static constexpr int TMEM_COLS = 512;
-  static_assert(2 * BN + NQT * D + (SEP_P ? NQT * BN / 2 : 0) <= TMEM_COLS, "tensor memory budget");
+  static_assert(2 * BN + NQT * D + (SEP_P ? NQT * BN / 2 : 0) + (Q_TMEM ? D / 2 : 0) <= TMEM_COLS,
+                "tensor memory budget");
   // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done, o_final[2], drain,
   // s_free[2], p_free[2], sched_full[SCHED], sched_empty[SCHED]
   static constexpr int SCHED = 4;  // units the producer may claim ahead of the consumers
@@ -262,7 +268,20 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     for (int kk = 0; kk < D / 16; ++kk) {
       const uint32_t ao = (kk / C::KPC) * C::Q_CHUNK_BYTES + (kk % C::KPC) * 32;
       const uint32_t bo = (kk / C::KPC) * C::KV_CHUNK_BYTES + (kk % C::KPC) * 32;
-      umma_ss(tmem + s_col, a0 + (ao >> 4), b0 + (bo >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+      if (C::Q_TMEM)
+        umma_ts(tmem + s_col, tmem + C::Q_COL + kk * 8, b0 + (bo >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+      else
+        umma_ss(tmem + s_col, a0 + (ao >> 4), b0 + (bo >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+    }
+  };
+  // Q tile -> TMEM (one 128-row x 16-element block per k-step, from the same shared-memory
+  // descriptor the QK would read it through). tcgen05.cp and tcgen05.mma issued by one thread run
+  // in issue order, so the copy lands after the previous unit's last QK and before this unit's.
+  auto copy_q_to_tmem = [&]() {
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint32_t ao = (kk / C::KPC) * C::Q_CHUNK_BYTES + (kk % C::KPC) * 32;
+      tmem_cp_128x256b(tmem + C::Q_COL + kk * 8, dQ + (ao >> 4));
     }
   };
   // O += P V over the tile's keys: A = P (bf16, in TMEM over S), B = V tile read MN-major (N = d),
@@ -377,6 +396,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         if (n == 0) continue;
         ok = mbar_wait(q_full, qc & 1, abort_flag, T);
         ++qc;
+        if (C::Q_TMEM && ok) {
+          copy_q_to_tmem();
+          umma_commit(q_empty);  // shared-memory Q is free once the copy is done
+        }
         const int base = pos;  // K_j at base + 2j, V_j at base + 2j + 1
         if (C::SEP_P) {
           // Two query tiles, P in buffers of its own. QK(t, j+1) may overwrite S once the softmax has
@@ -473,7 +496,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             if (!ok) break;
             issue_qk(0, ((t0 + j) & 1) ? C::S_COL1 : C::S_COL0, kv_slot(base + 2 * j));
             umma_commit(&s_full[(t0 + j) & 1]);
-            if (j == n - 1) umma_commit(q_empty);  // the unit's last QK: Q may be reloaded
+            if (!C::Q_TMEM && j == n - 1) umma_commit(q_empty);  // the unit's last QK: Q may be reloaded
             umma_commit(&kv_empty[kv_slot(base + 2 * j)]);
           }
           for (int j = 0; j < n && ok; ++j) {
@@ -493,7 +516,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               if (!ok) break;
               issue_qk(0, s_col, kv_slot(kp));
               umma_commit(&s_full[slot]);
-              if (j + 3 == n) umma_commit(q_empty);  // the unit's last QK
+              if (!C::Q_TMEM && j + 3 == n) umma_commit(q_empty);  // the unit's last QK
               umma_commit(&kv_empty[kv_slot(kp)]);
             }
           }
