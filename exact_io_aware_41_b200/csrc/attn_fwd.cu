@@ -36,6 +36,12 @@
 
 namespace attn {
 
+// K/V bytes of a whole launch below which all heads form one L2 group (see launch_fwd).
+#ifndef ATTN_L2_ONE_GROUP_MB
+#define ATTN_L2_ONE_GROUP_MB 96
+#endif
+constexpr double kL2OneGroupBytes = ATTN_L2_ONE_GROUP_MB * 1.0e6;
+
 // Running-max slack before O is rescaled, in log2 units: P entries stay <= 2^TAU.
 constexpr float kRescaleTau = 8.0f;
 
@@ -439,6 +445,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               tc_fence_after();
               issue_pv(qt ? C::O_COL1 : C::O_COL0, qt ? C::P_COL1 : C::P_COL0, kv_slot(pv_pos), j > 0);
               umma_commit(&p_free[qt]);
+              if (qt == 0 && j == nt[0] - 1 && nt[0] < n) umma_commit(&o_final[0]);  // see below
             }
             if (!ok) break;
             umma_commit(&kv_empty[kv_slot(pv_pos)]);
@@ -475,6 +482,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               ++pc[qt];
               tc_fence_after();
               issue_pv(qt ? C::O_COL1 : C::O_COL0, s_col, kv_slot(pv_pos), j > 0);
+              if (qt == 0 && j == nt[0] - 1 && nt[0] < n) umma_commit(&o_final[0]);  // see below
               // P of this tile is consumed by the PV MMAs above before this QK overwrites the slot:
               // MMAs issued by one thread execute in issue order.
               if (j + 1 < nt[qt]) {
@@ -524,9 +532,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           pos = base + 2 * n;
         }
         if (!ok) break;
-        // every MMA of this unit done: O may be read (one o_final per tile). (Q was released after the
-        // unit's last QK, so the next unit's Q load overlaps the last PVs and the epilogue.)
-        umma_commit(&o_final[0]);
+        // O may be read once every MMA writing it is done (one o_final phase per tile and unit), here
+        // after the unit's last PV. When tile 0 needs fewer K/V tiles (causal) its phase came right
+        // after its own last PV instead, so its epilogue runs during tile 1's last step. (Q was
+        // released after the unit's last QK, so the next unit's Q load overlaps the last PVs and the
+        // epilogues.)
+        if (C::NQT == 1 || un.n_tile0 == 0 || un.n_tile0 == n) umma_commit(&o_final[0]);
         if (C::NQT == 2) umma_commit(&o_final[1]);
       }
       if (!ok) {
@@ -816,10 +827,14 @@ static attn_status_t launch_fwd(const void* q, const void* k, const void* v, voi
   a.scale_log2 = scale * 1.4426950408889634f;
   a.timeout_ns = kWaitLimitNs;
   // heads per L2 group: K/V of one kv head is read by every query head of its group and block; keep
-  // a group's K/V within ~48 MB of the 126 MB L2
+  // a group's K/V within ~48 MB of the 126 MB L2. Causal launches whose K/V fits in L2 comfortably
+  // use one group: longest-first then runs over every unit, so no group's long units start near the
+  // end of the launch.
   {
     const double kv_bytes_per_head = 2.0 * Nkv * D * 2 / double(Hq / Hkv);
-    long long gh = (long long)(48.0e6 / kv_bytes_per_head);
+    const double kv_bytes_total = 2.0 * Nkv * D * 2 * double(B) * Hkv;
+    long long gh = (causal && kv_bytes_total <= kL2OneGroupBytes) ? (long long)B * Hq
+                                                                  : (long long)(48.0e6 / kv_bytes_per_head);
     if (gh < 1) gh = 1;
     if (gh > (long long)B * Hq) gh = (long long)B * Hq;
     a.heads_per_group = int(gh);
