@@ -627,20 +627,32 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           for (int i = 0; i < C::BN; ++i)
             if (kbase + i > lim) r[i] = __float_as_uint(-INFINITY);
         }
-        // row max: eight independent chains of 3-input max, then a short tree
+        // row max: a balanced tree of 3-input max (depth 5 for 128 keys; eight chains of 3-input
+        // max would be depth 9, and the first exponential waits for this max)
         float mx;
         {
-          constexpr int Q8 = C::BN / 8;
-          float m8[8];
+          float t[C::BN];
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            float a = __uint_as_float(r[kk * Q8]);
+          for (int i = 0; i < C::BN; ++i) t[i] = __uint_as_float(r[i]);
+          int m = C::BN;  // values left: t[0 .. m)
 #pragma unroll
-            for (int i = 1; i + 1 < Q8; i += 2)
-              a = fmax3(a, __uint_as_float(r[kk * Q8 + i]), __uint_as_float(r[kk * Q8 + i + 1]));
-            m8[kk] = (Q8 % 2 == 0) ? fmaxf(a, __uint_as_float(r[kk * Q8 + Q8 - 1])) : a;
+          for (int lvl = 0; lvl < 6; ++lvl) {  // 128 -> 44 -> 16 -> 6 -> 2 -> 1
+            if (m <= 1) break;
+            if (m == 2) {
+              t[0] = fmaxf(t[0], t[1]);
+              m = 1;
+              break;
+            }
+            const int n3 = m / 3, rem = m - 3 * n3;
+#pragma unroll
+            for (int i = 0; i < C::BN / 3 + 1; ++i)
+              if (i < n3) t[i] = fmax3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+              if (i < rem) t[n3 + i] = t[3 * n3 + i];
+            m = n3 + rem;
           }
-          mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+          mx = t[0];
         }
         const float m_new = fmaxf(m_ref, mx);
         // true when the max moved by more than TAU (also on the first live tile: -inf -> finite)

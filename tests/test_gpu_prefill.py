@@ -76,6 +76,39 @@ def test_small_head_dims_rescale_and_units_per_cta(lib, d):
     _run_small(lib, 4310 + d, 4, 16, 4, 1300, 1300, d, True, scale=0.6)
 
 
+DOMINANT_KEYS = (0, 63, 64, 100, 127, 128, 191, 255)  # first, middle and last of 64- and 128-key tiles
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_dominant_score_anywhere_in_a_tile(lib, d):
+    # Row i's score for key DOMINANT_KEYS[i % 8] is ~500 log2 units above every other score of the
+    # row, so every position of the key tiles holds some row's maximum. A row max that misses one
+    # position would leave 2^(score - max) to overflow; O must come out as that key's V row.
+    import torch
+
+    N = 256
+    qb, kb, vb = draw_prefill(4400 + d, 1, 1, 1, N, N, d)
+    q = synth.bf16_bits_to_f64(qb) * 0.01
+    k = synth.bf16_bits_to_f64(kb) * 0.01
+    big = 64.0
+    for m, key in enumerate(DOMINANT_KEYS):
+        k[0, key, 0, :8] = 0.0
+        k[0, key, 0, m] = big
+    for i in range(N):
+        q[0, i, 0, i % 8] = big
+    qb2, kb2 = synth.f64_to_bf16_bits(q), synth.f64_to_bf16_bits(k)
+    sc = 1.0 / math.sqrt(d)
+    o, lse = lib.attn_fwd(to_torch_bf16(qb2), to_torch_bf16(kb2), to_torch_bf16(vb), scale=sc, causal=False)
+    torch.cuda.synchronize()
+    O_ref, L_ref = oracle.attention(synth.bf16_bits_to_f64(qb2), synth.bf16_bits_to_f64(kb2),
+                                    synth.bf16_bits_to_f64(vb), sc, False)
+    og = bf16_tensor_to_f64(o)
+    lg = lse.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(og)) and np.all(np.isfinite(lg))
+    assert_parity(og, lg.transpose(0, 2, 1), O_ref, L_ref.transpose(0, 2, 1), f"dominant keys d{d}")
+    assert lib.attn_get_last_error() == lib.ATTN_OK
+
+
 def test_repeat_calls_are_identical(lib):
     import torch
 
