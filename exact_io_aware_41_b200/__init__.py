@@ -38,6 +38,7 @@ SIGNATURES = {
     "attn_status_string": (ctypes.c_char_p, [_I]),
     "attn_kernel_name": (ctypes.c_char_p, [_I]),
     "attn_selftest_bounded_wait": (_I, [ctypes.c_uint, _P]),
+    "attn_selftest_exp2_poly": (_I, [_P, _P, _I, _P]),
 }
 
 
@@ -218,3 +219,16 @@ def attn_get_last_error() -> int:
 
 def attn_selftest_bounded_wait(limit_us: int, stream=None) -> None:
     _check("attn_selftest_bounded_wait", lib_handle().attn_selftest_bounded_wait(int(limit_us), _stream(stream)))
+
+
+def attn_selftest_exp2_poly(x, out=None, stream=None):
+    """2^x through the library's FMA-pipe exponential, for a contiguous fp32 CUDA tensor x."""
+    import torch
+
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous() or x.numel() < 1:
+        raise ValueError("x must be a non-empty contiguous fp32 CUDA tensor")
+    if out is None:
+        out = torch.empty_like(x)
+    _check("attn_selftest_exp2_poly",
+           lib_handle().attn_selftest_exp2_poly(x.data_ptr(), out.data_ptr(), x.numel(), _stream(stream)))
+    return out

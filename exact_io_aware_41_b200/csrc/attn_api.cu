@@ -22,6 +22,19 @@ __global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns) {
   __syncthreads();
 }
 
+// 2^x through the FMA-pipe polynomial (exp2_poly2), two values per thread, for checking it against
+// the exact function.
+__global__ void exp2_poly_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int pairs = (n + 1) / 2;
+  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < pairs; p += gridDim.x * blockDim.x) {
+    const int i = 2 * p;
+    const bool two = i + 1 < n;
+    const float2 r = exp2_poly2(make_float2(x[i], two ? x[i + 1] : 0.f));
+    y[i] = r.x;
+    if (two) y[i + 1] = r.y;
+  }
+}
+
 // ---- driver entry point for cuTensorMapEncodeTiled (no link-time dependency on libcuda) ----
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -161,6 +174,15 @@ const char* attn_kernel_name(int which) {
 attn_status_t attn_selftest_bounded_wait(unsigned int limit_us, cudaStream_t stream) {
   if (limit_us == 0 || limit_us > 10000000u) return ATTN_ERR_INVALID_ARG;
   bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(1000ull * limit_us);
+  return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
+}
+
+attn_status_t attn_selftest_exp2_poly(const float* x, float* y, int n, cudaStream_t stream) {
+  if (!x || !y || n < 1) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) & 3u) || (reinterpret_cast<uintptr_t>(y) & 3u)) return ATTN_ERR_INVALID_ARG;
+  const long long pairs = (n + 1ll) / 2;
+  const int grid = int(pairs / 256 + 1 < 4096 ? pairs / 256 + 1 : 4096);
+  exp2_poly_selftest_kernel<<<grid, 256, 0, stream>>>(x, y, n);
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
 }
 

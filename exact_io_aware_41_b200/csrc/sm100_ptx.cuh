@@ -313,6 +313,30 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return d;
 }
 
+// 2^x for a pair, on the FMA pipe (x < 127.5, so that 2^n stays a normal float; the softmax's
+// arguments are at most TAU). Cody-Waite range reduction: x = n + f with
+// n = round(x) (the 1.5 * 2^23 addition rounds to an integer held in the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f by a degree-3 polynomial whose coefficients come from a relative-error
+// Remez fit (fit_exp2_poly.py beside this file, max relative error 7.5e-5); 2^n is added to the
+// exponent field. Inputs below -125 are clamped there (2^-125 instead of a smaller value).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f, c2 = 0.2426111251115799f,
+                  c3 = 0.0551716685295105f;
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);
+  float2 q = ffma2(make_float2(c3, c3), f, make_float2(c2, c2));
+  q = ffma2(q, f, make_float2(c1, c1));
+  q = ffma2(q, f, make_float2(c0, c0));
+  float2 out;
+  out.x = __int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23));
+  out.y = __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23));
+  return out;
+}
+
 // Named barrier over one warpgroup (128 threads): plain sync, and sync with an AND of a predicate.
 __device__ __forceinline__ void wg_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
 __device__ __forceinline__ bool wg_all(bool v, int id) {

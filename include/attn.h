@@ -159,6 +159,16 @@ const char* attn_kernel_name(int which);
  */
 attn_status_t attn_selftest_bounded_wait(unsigned int limit_us, cudaStream_t stream);
 
+/*
+ * Test hook for the FMA-pipe exponential (Cody-Waite range reduction and a degree-3 polynomial;
+ * the "emulated exponentials" the FlashAttention generation comparison record describes for
+ * FA-4). The prefill kernels can evaluate part of their exponentials with it (a build option, off
+ * by default). Writes y[i] = 2^x[i] through that approximation for n device floats (x < 127.5;
+ * inputs below -125 give 2^-125 times the polynomial's value at 0). Max relative error 7.5e-5 on
+ * [-125, 127.5). x and y are 4-byte aligned device pointers, n >= 1; asynchronous on `stream`.
+ */
+attn_status_t attn_selftest_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
