@@ -419,37 +419,70 @@ def time_prefill(lib, w, dev, stream, peaks, reps=20, warm=5):
 
 
 def e2e_prefill(lib, P, q, k, v, stream, n):
-    """Host (pinned) -> device copies, attn_fwd, device -> host copies of O and LSE, per step."""
+    """Per step: host (pinned) -> device copies of that step's Q, K, V, attn_fwd, and device -> host
+    copies of its O and LSE. Steps are pipelined the way a serving loop would run them: three
+    streams (copy in, compute, copy out) and two buffer sets, so step i+1's inputs cross PCIe while
+    step i computes and step i-1's result comes back (the link is full duplex)."""
     import torch
 
     hq = q.cpu().pin_memory()
     hk = k.cpu().pin_memory()
     hv = v.cpu().pin_memory()
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ho = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-    hl = torch.empty((P.B, P.Hq, P.Nq), dtype=torch.float32).pin_memory()
+    dev_in = [tuple(torch.empty_like(t) for t in (q, k, v)) for _ in range(2)]
+    dev_out = [(torch.empty_like(q), torch.empty((P.B, P.Hq, P.Nq), dtype=torch.float32, device=q.device))
+               for _ in range(2)]
+    ho = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(2)]
+    hl = [torch.empty((P.B, P.Hq, P.Nq), dtype=torch.float32).pin_memory() for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    s_cmp = stream
+    # per buffer set: inputs landed, inputs consumed, outputs written, outputs read back
+    ev = [{name: torch.cuda.Event() for name in ("in_done", "in_free", "out_done", "out_free")} for _ in range(2)]
+    used = [False, False]
 
-    def one():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        o, lse = lib.attn_fwd(dq, dk, dv, scale=P.scale, causal=P.causal)
-        ho.copy_(o, non_blocking=True)
-        hl.copy_(lse, non_blocking=True)
+    def one(i):
+        b = i & 1
+        e = ev[b]
+        dq, dk, dv = dev_in[b]
+        o, lse = dev_out[b]
+        with torch.cuda.stream(s_in):
+            if used[b]:
+                s_in.wait_event(e["in_free"])
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            e["in_done"].record(s_in)
+        s_cmp.wait_event(e["in_done"])
+        if used[b]:
+            s_cmp.wait_event(e["out_free"])
+        lib.attn_fwd(dq, dk, dv, scale=P.scale, causal=P.causal, out=o, lse=lse, stream=s_cmp)
+        e["in_free"].record(s_cmp)
+        e["out_done"].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(e["out_done"])
+            ho[b].copy_(o, non_blocking=True)
+            hl[b].copy_(lse, non_blocking=True)
+            e["out_free"].record(s_out)
+        used[b] = True
 
-    for _ in range(2):
-        one()
+    for i in range(2):
+        one(i)
     torch.cuda.synchronize()
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(n):
-        one()
-    b.record(stream)
-    b.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(s_in)  # every timed copy and launch is ordered after it through the events above
+    s_cmp.wait_event(start)
+    s_out.wait_event(start)
+    for i in range(n):
+        one(i)
+    end_cmp = torch.cuda.Event()
+    end_cmp.record(s_cmp)
+    s_out.wait_event(end_cmp)
+    with torch.cuda.stream(s_out):
+        s_out.wait_stream(s_in)
+        end.record(s_out)
+    end.synchronize()
     h2d = 3 * q.numel() * 2
     d2h = q.numel() * 2 + P.B * P.Hq * P.Nq * 4
-    return {"ms": a.elapsed_time(b) / n, "h2d": h2d, "d2h": d2h}
+    return {"ms": start.elapsed_time(end) / n, "h2d": h2d, "d2h": d2h}
 
 
 def e2e_decode(lib, Dw, dq, kc, vc, lens_np, stream, n):
