@@ -43,9 +43,9 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 # in profiles/), keyed to the sha256 of the kernel's source file it was measured on: once that file
 # changes, the figure is stale and the bench line reports null until it is measured again.
 NCU_TRAFFIC = {
-    # attn_fwd_kernel<128> on the causal B4 H16 N2048 d128 workload: 125.47 MB read + 10.72 MB written
+    # attn_fwd_kernel<128> on the causal B4 H16 N2048 d128 workload: 129.30 MB read + 11.46 MB written
     "prefill": ("exact_io_aware_41_b200/csrc/attn_fwd.cu",
-                "15a79acdd8aa6692c9a6700de4fa324d01d0cd0a41797a61b249402d292c4f72", 136_189_696.0),
+                "d7831d457b958eb1db8bf4ad34c593d29c3ad3a88ef0f957d626865c180d3ee5", 140_756_224.0),
     # decode_split_tc_kernel<128,4> (2123.74 MB read + 7.08 MB written) + decode_combine_kernel<128>
     # (4.29 MB read) on the full decode workload
     "decode": ("exact_io_aware_41_b200/csrc/attn_decode.cu",

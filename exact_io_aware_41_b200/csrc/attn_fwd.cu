@@ -1,31 +1,33 @@
 // Prefill forward for sm_100a: O = softmax(scale * Q K^T) V and LSE, tile by tile.
 //
-// Work decomposition (one CTA per unit): a unit is (batch b, query head h, block of NQT query
-// tiles of 128 rows). Units are numbered so the block scheduler hands out the heaviest causal units
-// first (longest-processing-time order). Query-block parallelism follows the "FlashAttention
-// evolution" article, section 3; LPT ordering the FlashAttention generation comparison record,
-// "Workarounds" (FA-4).
+// Work decomposition: a unit is (batch b, query head h, block of NQT query tiles of 128 rows). The
+// grid is persistent (one CTA per SM); each CTA claims units from a per-launch atomic counter.
+// Units are numbered by L2 head group and, inside a group, heaviest first (longest-processing-time
+// order for causal masks). Query-block parallelism follows the "FlashAttention evolution" article,
+// section 3; LPT ordering the FlashAttention generation comparison record, "Workarounds" (FA-4).
 //
 // Roles inside a CTA (warp specialisation, evolution article section 4, rebuilt on sm_100a):
-//   warp 0        TMA producer: Q tiles once, then K_j, V_j into a STAGES-deep shared-memory ring
+//   warp 0        TMA producer: claims units, loads each unit's Q tiles once, then K_j, V_j into a
+//                 STAGES-deep shared-memory ring
 //   warp 1        MMA issuer (one thread): S = Q K^T and O += P V with tcgen05.mma, accumulators
 //                 in tensor memory (evolution article section 5)
 //   warp 2        tensor-memory allocator
 //   warpgroups 1+ softmax: each thread owns one query row = one TMEM lane ("sliced-Q" ownership,
 //                 section 3, so no cross-thread reduction). Reads S from TMEM, applies the mask,
-//                 runs the online-softmax update, writes P (bf16) back over S for the PV MMA, and
+//                 runs the online-softmax update, writes P (bf16) to TMEM for the PV MMA, and
 //                 rescales O in TMEM only when its running max grew by more than TAU (conditional
 //                 rescaling, section 5). At the end it divides by the row sum once (delayed
 //                 normalisation, section 3) and writes O and LSE.
 // With two query tiles per CTA (d <= 128) the two softmax warpgroups alternate with the tensor
 // core: while one tile's softmax runs, the other tile's MMAs run ("overlaps multiple query tiles",
-// section 5). With d = 256 one query tile alternates between two S buffers instead.
+// section 5). With d = 256 one query tile alternates between two S buffers instead, and its Q tile
+// is copied into TMEM once per unit so the QK MMAs read only K from shared memory.
 //
 // S and P never leave the SM: S is fp32 in TMEM, P is bf16 in TMEM, read by the MMA straight from
-// there. At d = 128 (and 256) P is written in place over S, so a tile's next S = Q K^T waits for
-// the PV that reads P. At d <= 64 the O accumulators are narrow enough to leave TMEM columns for
-// P buffers of its own: the next S of a tile is computed as soon as the softmax has read the
-// current one, overlapping that tile's own softmax.
+// there. At d = 128 and 256 P is written in place over S, so the next S = Q K^T into that slot
+// waits for the PV that reads P. At d <= 64 the O accumulators are narrow enough to leave TMEM
+// columns for P buffers of its own: the next S of a tile is computed as soon as the softmax has
+// read the current one, overlapping that tile's own softmax.
 #include <cuda_bf16.h>
 #include <math.h>
 
