@@ -2,14 +2,16 @@
 """Benchmark of the exact-attention hot path on B200; prints one JSON line on rank 0.
 
 A step is one pass over both entry points of the hot path:
-  * prefill: attn_fwd on the causal workload B=4, H=16, N=2048, d=128 (bf16, scale 1/sqrt(d));
+  * prefill: attn_fwd on the long non-causal workload B=2, H=16, N=8192, d=128 (bf16, scale
+             1/sqrt(d)), the configuration the >=60 % tensor-core gate is stated on;
   * decode:  attn_decode_splitkv (split kernel + combine) on B=8, Hq=32, Hkv=8, d=128 with KV
              lengths drawn uniformly from [1024, 131072].
-`value` is the prefill throughput in TFLOP/s (causal FLOPs = half of 4*B*H*N^2*d); the decode half
-of the metric is reported under "decode" in GB/s of algorithmic HBM bytes. Both are timed with CUDA
-events on the launching stream; the step's inputs (2.3 GB) exceed the 126 MB L2, and the decode pass
-evicts the prefill inputs before the next step. "gates" times the long-sequence prefill workloads
-(N=8192) and the head-dim sweep the same way.
+`value` is the prefill throughput in TFLOP/s (4*B*H*N^2*d); the decode half of the metric is
+reported under "decode" in GB/s of algorithmic HBM bytes. Both are timed with CUDA events on the
+launching stream; the step's inputs (0.2 GB prefill + 4.3 GB decode) exceed the 126 MB L2, and the
+decode pass evicts the prefill inputs before the next step. "gates" times the other prefill
+workloads (causal N=2048, causal and GQA N=8192, the head-dim sweep) one launch at a time with a
+256 MiB L2 flush before each.
 
 `--impl reference` times the CPU oracle instead, on a bounded sample of the same workloads.
 Multi-GPU (torchrun): every rank runs the same step on its own GPU (independent problems, no
@@ -40,23 +42,24 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 
 
 # DRAM traffic per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum; summaries and commands
-# in profiles/), keyed to the sha256 of the kernel's source file it was measured on: once that file
-# changes, the figure is stale and the bench line reports null until it is measured again.
+# in profiles/), per workload, keyed to the sha256 of the kernel source it was measured on: once
+# that file changes, the figure is stale and the bench line reports null until it is measured again.
+PREFILL_SRC = "exact_io_aware_41_b200/csrc/attn_fwd.cu"
+DECODE_SRC = "exact_io_aware_41_b200/csrc/attn_decode.cu"
 NCU_TRAFFIC = {
-    # attn_fwd_kernel<128> on the causal B4 H16 N2048 d128 workload: 129.30 MB read + 11.46 MB written
-    "prefill": ("exact_io_aware_41_b200/csrc/attn_fwd.cu",
-                "d7831d457b958eb1db8bf4ad34c593d29c3ad3a88ef0f957d626865c180d3ee5", 140_756_224.0),
     # decode_split_tc_kernel<128,4> (2123.74 MB read + 7.08 MB written) + decode_combine_kernel<128>
     # (4.29 MB read) on the full decode workload
-    "decode": ("exact_io_aware_41_b200/csrc/attn_decode.cu",
-               "8f7ae30438212f2aa0baa6b8c3896abe248dbfb72e17985d9f09ab0e1293ef52", 2_135_109_632.0),
+    synth.DECODE.name: (DECODE_SRC, "8f7ae30438212f2aa0baa6b8c3896abe248dbfb72e17985d9f09ab0e1293ef52",
+                        2_135_109_632.0),
 }
 
 
-def ncu_traffic(kind: str):
+def ncu_traffic(name: str):
     import hashlib
 
-    path, digest, nbytes = NCU_TRAFFIC[kind]
+    if name not in NCU_TRAFFIC:
+        return None
+    path, digest, nbytes = NCU_TRAFFIC[name]
     try:
         with open(os.path.join(ROOT, path), "rb") as f:
             return nbytes if hashlib.sha256(f.read()).hexdigest() == digest else None
@@ -213,24 +216,30 @@ def cpu_prefill(w: synth.Prefill, budget_s: float):
     return flops / spent / 1e12, f"{heads} of {w.B * w.Hq} (b, h) heads of {w.name}, {spent:.1f} s", spent
 
 
-def cpu_decode(w: synth.Decode, budget_s: float, tokens: int = 16384):
-    """Oracle decode on batch row 0 truncated to `tokens` KV tokens, repeated until the budget is spent."""
+def cpu_decode(w: synth.Decode, budget_s: float, tokens: int = 2048):
+    """Oracle decode on all B sequences and all query heads, each sequence truncated to its first
+    `tokens` KV tokens (host draws of the same seeded cache), repeated until the budget is spent."""
     import oracle
 
-    L = min(tokens, int(w.lengths()[0]))
-    cap = L
-    shape = (1, cap, w.Hkv, w.d)
-    q = synth.bf16_bits_to_f64(synth.normal_bf16(w.seed, synth.STREAM_Q, (1, w.Hq, w.d)))
-    k = synth.bf16_bits_to_f64(synth.normal_bf16(w.seed, synth.STREAM_K, shape))
-    v = synth.bf16_bits_to_f64(synth.normal_bf16(w.seed, synth.STREAM_V, shape))
+    lens = np.minimum(w.lengths(), tokens)
+    cap = int(lens.max())
+    shape = (w.B, cap, w.Hkv, w.d)
+    q = synth.bf16_bits_to_f64(synth.normal_bf16(w.seed, synth.STREAM_Q, (w.B, w.Hq, w.d)))
+    # the first `cap` tokens of the full cache [B, Nkv_cap, Hkv, d]: draw those rows of each sequence
+    row = np.arange(cap * w.Hkv * w.d, dtype=np.int64)
+    flat = (np.arange(w.B, dtype=np.int64)[:, None] * (w.cap * w.Hkv * w.d) + row[None, :]).reshape(-1)
+    k = synth.bf16_bits_to_f64(synth.normal_bf16_at(w.seed, synth.STREAM_K, flat)).reshape(shape)
+    v = synth.bf16_bits_to_f64(synth.normal_bf16_at(w.seed, synth.STREAM_V, flat)).reshape(shape)
+    per_rep = int(lens.astype(np.int64).sum()) * w.Hkv * w.d * 2 * 2
     byts, spent, reps = 0.0, 0.0, 0
     while spent < budget_s:
         t0 = time.perf_counter()
-        oracle.decode(q, k, v, np.array([L]), w.scale)
+        oracle.decode(q, k, v, lens, w.scale)
         spent += time.perf_counter() - t0
-        byts += L * w.Hkv * w.d * 2 * 2
+        byts += per_rep
         reps += 1
-    return byts / spent / 1e9, f"{reps} x (batch row 0, first {L} KV tokens, all {w.Hq} heads) of {w.name}", spent
+    return byts / spent / 1e9, (f"{reps} x (all {w.B} sequences truncated to their first {tokens} KV tokens, "
+                                f"all {w.Hq} query heads) of {w.name}"), spent
 
 
 # ------------------------------------------------------------------------------------------------
@@ -246,7 +255,7 @@ def run_ours(args, world, rank, local, dist):
     stream = torch.cuda.current_stream()
     peaks, peak_src = _peaks()
 
-    P = synth.CAUSAL_2K
+    P = synth.LONG_8K
     Dw = synth.DECODE
     q = synth.normal_bf16_torch(P.seed, synth.STREAM_Q, (P.B, P.Nq, P.Hq, P.d), dev)
     k = synth.normal_bf16_torch(P.seed, synth.STREAM_K, (P.B, P.Nkv, P.Hkv, P.d), dev)
@@ -316,11 +325,10 @@ def run_ours(args, world, rank, local, dist):
     dec_gbs_1 = dec_bytes / dec_avg_s / 1e9
     dec_value = world * K * dec_bytes / (dec_ms * 1e-3) / 1e9
 
-    # ---- gates: long-sequence prefill and head-dim sweep (same timing, not part of `value`)
+    # ---- gates: the other prefill workloads, one launch at a time after an L2 flush (not in `value`)
     gates = {}
     if not args.no_gates:
-        for w in (synth.LONG_8K, synth.LONG_8K_CAUSAL, synth.LONG_8K_GQA, synth.LONG_8K_GQA_CAUSAL,
-                  *synth.SWEEP):
+        for w in GATES:
             gates[w.name] = time_prefill(lib, w, dev, stream, peaks)
             torch.cuda.empty_cache()
 
@@ -361,13 +369,15 @@ def run_ours(args, world, rank, local, dist):
             "decode_workload": Dw.name,
             "decode_kv_tokens": int(lens_np.sum()),
             "parallelism": f"replica x{world} (independent problems, no collective)",
-            "l2": "inputs larger than L2: the step reads 2.3 GB; the decode pass evicts the prefill inputs",
+            "l2": "inputs larger than L2: the step reads 4.5 GB (prefill 0.2 GB); the decode pass evicts the "
+                  "prefill inputs; gates flush L2 (256 MiB write) before every launch",
         },
         "frac_of_nominal_bf16": pf_tflops_1 / NOMINAL_BF16_TFLOPS,
         "roofline": {"bound": "tensor", "kernel": lib.kernel_name(0).replace("<D>", "<128>"),
                      "achieved": pf_tflops_1, "peak": meas_tf, "unit": "TFLOP/s", "frac": pf_tflops_1 / meas_tf,
                      "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
-                     "traffic": args.prefill_traffic if args.prefill_traffic is not None else ncu_traffic("prefill")},
+                     "traffic": ncu_traffic(P.name), "traffic_source": "ncu dram__bytes_read.sum + "
+                     "dram__bytes_write.sum of one launch on this workload (null: not measured on this source)"},
         "decode": {
             "value": dec_value, "unit": "GB/s", "ms_per_call": dec_avg_s * 1e3,
             "algorithmic_bytes_per_call": dec_bytes,
@@ -375,7 +385,7 @@ def run_ours(args, world, rank, local, dist):
             "roofline": {"bound": "hbm", "kernel": "decode_split_tc_kernel<128,4> + decode_combine_kernel<128>",
                          "achieved": dec_gbs_1, "peak": meas_bw, "unit": "GB/s", "frac": dec_gbs_1 / meas_bw,
                          "peak_source": f"{peak_src} copy bandwidth",
-                         "traffic": args.decode_traffic if args.decode_traffic is not None else ncu_traffic("decode")},
+                         "traffic": ncu_traffic(Dw.name)},
             "e2e": dec_e2e and {
                 "value": world * dec_bytes / (dec_e2e["ms"] * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": dec_e2e["h2d"], "d2h_bytes_per_step": dec_e2e["d2h"]},
@@ -389,6 +399,15 @@ def run_ours(args, world, rank, local, dist):
         "cpu_baseline": cpu,
     }
     return line
+
+
+GATES = (synth.CAUSAL_2K, synth.LONG_8K_CAUSAL, synth.LONG_8K_GQA, synth.LONG_8K_GQA_CAUSAL, *synth.SWEEP)
+
+
+def prefill_bytes(w) -> int:
+    """Algorithmic HBM bytes of one prefill launch: Q, K, V read once, O and LSE written once."""
+    return (2 * w.B * w.Nq * w.Hq * w.d + 2 * 2 * w.B * w.Nkv * w.Hkv * w.d + 2 * w.B * w.Nq * w.Hq * w.d
+            + 4 * w.B * w.Hq * w.Nq)
 
 
 def time_prefill(lib, w, dev, stream, peaks, reps=20, warm=5):
@@ -414,8 +433,11 @@ def time_prefill(lib, w, dev, stream, peaks, reps=20, warm=5):
         ms.append(a.elapsed_time(b))
     med = float(np.median(ms))
     tf = w.flops / (med * 1e-3) / 1e12
-    return {"ms": med, "tflops": tf, "frac_of_measured": tf / peaks.get("bf16_tflops", FALLBACK["bf16_tflops"]),
-            "frac_of_nominal": tf / NOMINAL_BF16_TFLOPS}
+    pk = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
+    return {"ms": med, "tflops": tf, "frac_of_measured": tf / pk, "frac_of_nominal": tf / NOMINAL_BF16_TFLOPS,
+            "roofline": {"bound": "tensor", "kernel": f"attn::attn_fwd_kernel<{w.d}>", "achieved": tf, "peak": pk,
+                         "unit": "TFLOP/s", "frac": tf / pk, "traffic": ncu_traffic(w.name),
+                         "algorithmic_bytes": prefill_bytes(w)}}
 
 
 def e2e_prefill(lib, P, q, k, v, stream, n):
@@ -550,9 +572,9 @@ def run_reference(args, world, rank):
 
     if rank != 0:
         return None
-    P, Dw = synth.CAUSAL_2K, synth.DECODE
+    P, Dw = synth.LONG_8K, synth.DECODE
     m = 64
-    blocks = [(b, h, i0) for (b, h) in ((0, 0), (1, 5), (2, 10), (3, 15)) for i0 in range(0, P.Nq, m)]
+    blocks = [(b, h, i0) for (b, h) in ((0, 0), (1, 5), (0, 10), (1, 15)) for i0 in range(0, P.Nq, m)]
     per_step = min(1.0, 100.0 / max(1, args.steps))  # keeps K steps within a couple of minutes
     cursor = 0
 
@@ -611,7 +633,7 @@ def run_only(args):
     peaks, src = _peaks()
     if args.only == "prefill":
         table = {w.name: w for w in synth.PREFILL_WORKLOADS}
-        w = table[args.workload] if args.workload else synth.CAUSAL_2K
+        w = table[args.workload] if args.workload else synth.LONG_8K
         q = synth.normal_bf16_torch(w.seed, synth.STREAM_Q, (w.B, w.Nq, w.Hq, w.d), dev)
         k = synth.normal_bf16_torch(w.seed, synth.STREAM_K, (w.B, w.Nkv, w.Hkv, w.d), dev)
         v = synth.normal_bf16_torch(w.seed, synth.STREAM_V, (w.B, w.Nkv, w.Hkv, w.d), dev)
@@ -668,9 +690,6 @@ def main():
     ap.add_argument("--no-gates", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e-decode", action="store_true")
-    ap.add_argument("--prefill-traffic", type=float, default=None,
-                    help="ncu dram bytes per prefill launch, when measured for the current kernel")
-    ap.add_argument("--decode-traffic", type=float, default=None)
     ap.add_argument("--only", choices=("prefill", "decode"), default=None,
                     help="time one kernel on one workload (profiling and per-workload numbers)")
     ap.add_argument("--workload", default=None, help="prefill workload name for --only prefill")

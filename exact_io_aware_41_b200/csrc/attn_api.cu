@@ -1,6 +1,7 @@
 // The C ABI (include/attn.h): argument checks, TMA descriptors, launches, the device error word.
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <atomic>
 #include <mutex>
 
 #include "attn_internal.h"
@@ -49,25 +50,111 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-bool encode_tile_map(CUtensorMap* map, const void* base, int d, int heads, int rows, int outer, int box_cols,
-                     int box_rows, unsigned swizzle_bytes) {
+static bool encode_tile_map_uncached(CUtensorMap* map, const void* base, int d, int heads, int rows, int outer,
+                                     int box_cols, int box_rows, unsigned swizzle_bytes) {
   auto fn = get_encode_fn();
   if (fn == nullptr) return false;
   const cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(heads), cuuint64_t(rows), cuuint64_t(outer)};
   const cuuint64_t strides[3] = {cuuint64_t(d) * 2, cuuint64_t(heads) * d * 2, cuuint64_t(rows) * heads * d * 2};
   const cuuint32_t box[4] = {cuuint32_t(box_cols), 1u, cuuint32_t(box_rows), 1u};
   const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
-  const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
+namespace {
+// Recently encoded tensor maps, replaced round robin. Every field that enters the encoding is part
+// of the key, so a hit returns exactly the map the encoder would produce.
+struct MapKey {
+  const void* base;
+  int d, heads, rows, outer, box_cols, box_rows;
+  unsigned swizzle;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && d == o.d && heads == o.heads && rows == o.rows && outer == o.outer &&
+           box_cols == o.box_cols && box_rows == o.box_rows && swizzle == o.swizzle;
+  }
+};
+constexpr int kMapCacheSize = 64;
+struct MapCache {
+  std::mutex mu;
+  MapKey key[kMapCacheSize];
+  CUtensorMap map[kMapCacheSize];
+  bool used[kMapCacheSize] = {};
+  int next = 0;
+};
+MapCache& map_cache() {
+  static MapCache c;
+  return c;
+}
+}  // namespace
+
+bool encode_tile_map(CUtensorMap* map, const void* base, int d, int heads, int rows, int outer, int box_cols,
+                     int box_rows, unsigned swizzle_bytes) {
+  const MapKey k{base, d, heads, rows, outer, box_cols, box_rows, swizzle_bytes};
+  MapCache& c = map_cache();
+  std::lock_guard<std::mutex> lock(c.mu);
+  for (int i = 0; i < kMapCacheSize; ++i) {
+    if (c.used[i] && c.key[i] == k) {
+      *map = c.map[i];
+      return true;
+    }
+  }
+  if (!encode_tile_map_uncached(map, base, d, heads, rows, outer, box_cols, box_rows, swizzle_bytes)) return false;
+  const int slot = c.next;
+  c.next = (c.next + 1) % kMapCacheSize;
+  c.key[slot] = k;
+  c.map[slot] = *map;
+  c.used[slot] = true;
+  return true;
+}
+
+namespace {
+std::mutex g_attr_mu;
+// (function, device) -> dynamic shared memory bytes the function has been opted into
+struct AttrEntry {
+  const void* func;
+  int dev;
+  int bytes;
+};
+AttrEntry g_attr[512];
+int g_attr_n = 0;
+std::atomic<int> g_sm_count[kMaxDevices];
+}  // namespace
+
+cudaError_t ensure_dyn_smem(const void* func, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  int i = 0;
+  for (; i < g_attr_n; ++i)
+    if (g_attr[i].func == func && g_attr[i].dev == dev) break;
+  if (i < g_attr_n && g_attr[i].bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  if (i == g_attr_n) {
+    if (g_attr_n == int(sizeof(g_attr) / sizeof(g_attr[0]))) return cudaSuccess;  // table full: set every time
+    g_attr[g_attr_n++] = AttrEntry{func, dev, bytes};
+  } else {
+    g_attr[i].bytes = bytes;
+  }
+  return cudaSuccess;
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (dev >= 0 && dev < kMaxDevices) {
+    const int cached = g_sm_count[dev].load(std::memory_order_relaxed);
+    if (cached > 0) return cached;
+  }
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  if (dev >= 0 && dev < kMaxDevices) g_sm_count[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -112,12 +199,14 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
     return ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
   const int G = Hq / Hkv;
-  if ((d != 64 && d != 128 && d != 256) || (G != 1 && G != 2 && G != 4 && G != 8)) return ATTN_ERR_UNSUPPORTED;
+  if ((d != 32 && d != 64 && d != 128 && d != 256) || (G != 1 && G != 2 && G != 4 && G != 8))
+    return ATTN_ERR_UNSUPPORTED;
   if (chunk == 0) chunk = decode_default_chunk(B, Hkv, Nkv_cap);
   const long long n_splits = (Nkv_cap + (long long)chunk - 1) / chunk;
+  // every size check comes before the split kernel is enqueued, so a refused call leaves nothing behind
+  if (Hkv > 65535 || B > 65535 || !combine_fits(n_splits)) return ATTN_ERR_UNSUPPORTED;
   const size_t need = decode_workspace(B, Hq, d, Nkv_cap, chunk);
   if (workspace == nullptr || !is_aligned16(workspace) || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
-  if (Hkv > 65535 || B > 65535) return ATTN_ERR_UNSUPPORTED;
   float* po = static_cast<float*>(workspace);
   const size_t po_bytes = size_t(B) * Hq * n_splits * d * sizeof(float);
   float* pl = reinterpret_cast<float*>(static_cast<char*>(workspace) + ((po_bytes + 255) / 256) * 256);
@@ -135,7 +224,7 @@ attn_status_t attn_decode_combine(const float* part_o, const float* part_lse, in
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return ATTN_ERR_INVALID_ARG;
   if (rows < 1 || n_splits < 1) return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
+  if ((d != 32 && d != 64 && d != 128 && d != 256) || !combine_fits(n_splits)) return ATTN_ERR_UNSUPPORTED;
   return decode_combine_dispatch(part_o, part_lse, rows, n_splits, d, o, lse, stream);
 }
 

@@ -275,20 +275,31 @@ struct DecTcCfg {
   static constexpr int NW = 4;                  // consumer warps
   static constexpr int TT = 16 * NW;            // tokens per tile
   static constexpr int STAGES = 3;
-  static constexpr int NCHUNK = D / 64;         // 64-element (128-byte) swizzle chunks along d
-  static constexpr int CHUNK_BYTES = TT * 128;
+  // Rows of a tile are stored in chunks of CE elements along d: 64 elements (128 bytes) with the
+  // 128-byte swizzle for d >= 64; d = 32 uses plain 64-byte rows (no swizzle).
+  static constexpr int CE = D < 64 ? D : 64;
+  static constexpr int ROWB = CE * 2;           // bytes per stored row of a chunk
+  static constexpr bool SWIZZLE = (D >= 64);
+  static constexpr int NCHUNK = D / CE;
+  static constexpr int CHUNK_BYTES = TT * ROWB;
   static constexpr int TILE_BYTES = TT * D * 2;  // one K or V tile
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int THREADS = 32 * (NW + 1);
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 2 * STAGES * 8 + 16;
 };
 
-// Byte address of element (row, col) of a TT x D bf16 tile written by TMA with 128-byte swizzle:
-// 64-column chunks, 128-byte rows, the 16-byte unit index XOR-ed with the row index mod 8.
+// Byte address of element (row, col) of a TT x D bf16 tile written by TMA. With the 128-byte
+// swizzle (d >= 64): 64-column chunks of 128-byte rows, the 16-byte unit index XOR-ed with the row
+// index mod 8. Without (d = 32): one chunk of plain 64-byte rows.
 template <int D>
 __device__ __forceinline__ uint32_t dec_sw128(uint32_t tile, int row, int col) {
-  const int chunk = col >> 6, unit = (col & 63) >> 3;
-  return tile + chunk * DecTcCfg<D>::CHUNK_BYTES + row * 128 + ((unit ^ (row & 7)) << 4) + ((col & 7) << 1);
+  using C = DecTcCfg<D>;
+  if constexpr (C::SWIZZLE) {
+    const int chunk = col >> 6, unit = (col & 63) >> 3;
+    return tile + chunk * C::CHUNK_BYTES + row * 128 + ((unit ^ (row & 7)) << 4) + ((col & 7) << 1);
+  } else {
+    return tile + row * C::ROWB + (col << 1);
+  }
 }
 
 template <int D, int G>
@@ -347,8 +358,8 @@ __global__ void __launch_bounds__(DecTcCfg<D>::THREADS, 2)
         const int tok = t_begin + i * C::TT;
 #pragma unroll
         for (int c = 0; c < C::NCHUNK; ++c) {
-          tma_load_4d(kt + c * C::CHUNK_BYTES, &tmK, &full[st], c * 64, g, tok, b);
-          tma_load_4d(kt + C::TILE_BYTES + c * C::CHUNK_BYTES, &tmV, &full[st], c * 64, g, tok, b);
+          tma_load_4d(kt + c * C::CHUNK_BYTES, &tmK, &full[st], c * C::CE, g, tok, b);
+          tma_load_4d(kt + C::TILE_BYTES + c * C::CHUNK_BYTES, &tmV, &full[st], c * C::CE, g, tok, b);
         }
       }
       if (i < n_tiles) {
@@ -437,9 +448,11 @@ __global__ void __launch_bounds__(DecTcCfg<D>::THREADS, 2)
       // V rows past the end of the sequence may hold anything (0 * NaN would poison O): zero them
       if (valid < 16) {
         const int first = valid < 0 ? 0 : valid;
+        // whole rows are zeroed, so the swizzle (a permutation inside a row) does not matter
+        constexpr int UPR = C::ROWB / 16;  // 16-byte units per stored row of a chunk
         for (int idx = lane; idx < (16 - first) * (D / 8); idx += 32) {
           const int r = first + idx / (D / 8), unit = idx % (D / 8);
-          const uint32_t a = vt + (unit >> 3) * C::CHUNK_BYTES + (16 * warp + r) * 128 + ((unit & 7) << 4);
+          const uint32_t a = vt + (unit / UPR) * C::CHUNK_BYTES + (16 * warp + r) * C::ROWB + ((unit % UPR) << 4);
           asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(0u) : "memory");
         }
         __syncwarp();
@@ -504,11 +517,15 @@ __global__ void __launch_bounds__(DecTcCfg<D>::THREADS, 2)
 template <int D>
 struct CombCfg {
   static constexpr int NT = D <= 128 ? 32 : 64;  // threads per row
-  static constexpr int EPT = D / NT;             // elements per thread (2 or 4)
+  static constexpr int EPT = D / NT;             // elements per thread (1, 2 or 4)
 };
 
 template <int EPT>
 struct VecF;
+template <>
+struct VecF<1> {
+  static __device__ __forceinline__ void fma(float w, const float* src, float* acc) { acc[0] = fmaf(w, *src, acc[0]); }
+};
 template <>
 struct VecF<2> {
   using T = float2;
@@ -585,11 +602,16 @@ __global__ void __launch_bounds__(CombCfg<D>::NT)
   }
   const float inv = (z > 0.f) ? 1.0f / z : 0.f;
   __nv_bfloat16* orow = o + size_t(row) * D + t * EPT;
+  if constexpr (EPT == 1) {
+    const float a0 = (acc[0][0] + acc[1][0]) + (acc[2][0] + acc[3][0]);
+    orow[0] = __float2bfloat16_rn(a0 * inv);
+  } else {
 #pragma unroll
-  for (int e = 0; e < EPT; e += 2) {
-    const float a0 = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
-    const float a1 = (acc[0][e + 1] + acc[1][e + 1]) + (acc[2][e + 1] + acc[3][e + 1]);
-    *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16x2(a0 * inv, a1 * inv);
+    for (int e = 0; e < EPT; e += 2) {
+      const float a0 = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
+      const float a1 = (acc[0][e + 1] + acc[1][e + 1]) + (acc[2][e + 1] + acc[3][e + 1]);
+      *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16x2(a0 * inv, a1 * inv);
+    }
   }
   if (t == 0) lse[row] = (z > 0.f) ? mx + logf(z) : -INFINITY;
 }
@@ -600,7 +622,9 @@ __global__ void __launch_bounds__(CombCfg<D>::NT)
 int decode_default_chunk(int B, int Hkv, int Nkv_cap) {
   // aim for ~8 live CTAs per SM if every sequence were full, in multiples of 64 tokens, at most 2048
   const long long total = (long long)B * Hkv * Nkv_cap;
-  long long c = total / (148LL * 8);
+  int sms = sm_count();
+  if (sms <= 0) sms = 148;  // no device visible: size for a B200
+  long long c = total / (sms * 8LL);
   c = (c + 63) / 64 * 64;
   if (c < 64) c = 64;
   if (c > 2048) c = 2048;
@@ -632,16 +656,12 @@ static attn_status_t launch_split_tc(const void* q, const void* kc, const void* 
                                      cudaStream_t stream) {
   using C = DecTcCfg<D>;
   CUtensorMap tmK, tmV;
-  if (!encode_tile_map(&tmK, kc, D, Hkv, cap, B, 64, C::TT, 128) ||
-      !encode_tile_map(&tmV, vc, D, Hkv, cap, B, 64, C::TT, 128))
+  const unsigned swz = C::SWIZZLE ? 128u : 0u;
+  if (!encode_tile_map(&tmK, kc, D, Hkv, cap, B, C::CE, C::TT, swz) ||
+      !encode_tile_map(&tmV, vc, D, Hkv, cap, B, C::CE, C::TT, swz))
     return ATTN_ERR_CUDA;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(decode_split_tc_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_BYTES) != cudaSuccess)
-      return ATTN_ERR_CUDA;
-    attr_set = true;
-  }
+  if (ensure_dyn_smem(reinterpret_cast<const void*>(decode_split_tc_kernel<D, G>), C::SMEM_BYTES) != cudaSuccess)
+    return ATTN_ERR_CUDA;
   dim3 grid(n_splits, Hkv, B);
   decode_split_tc_kernel<D, G><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(
       tmK, tmV, reinterpret_cast<const __nv_bfloat16*>(q), lens, cap, Hkv, chunk, n_splits,
@@ -649,7 +669,7 @@ static attn_status_t launch_split_tc(const void* q, const void* kc, const void* 
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
 }
 
-// d = 64 and 128 use the tensor-core split kernel; d = 256 (whose O fragments would not fit the
+// d = 32, 64 and 128 use the tensor-core split kernel; d = 256 (whose O fragments would not fit the
 // register budget) uses the CUDA-core one.
 template <int D>
 static attn_status_t split_by_group(int G, const void* q, const void* kc, const void* vc, const int32_t* lens,
@@ -679,6 +699,7 @@ attn_status_t decode_split_dispatch(const void* q, const void* kc, const void* v
                                     float* po, float* pl, cudaStream_t st) {
   const int G = Hq / Hkv;
   switch (d) {
+    case 32: return split_by_group<32>(G, q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
     case 64: return split_by_group<64>(G, q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
     case 128: return split_by_group<128>(G, q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
     case 256: return split_by_group<256>(G, q, kc, vc, lens, cap, B, Hkv, chunk, n_splits, scale, po, pl, st);
@@ -686,28 +707,28 @@ attn_status_t decode_split_dispatch(const void* q, const void* kc, const void* v
   }
 }
 
+template <int D>
+static attn_status_t launch_combine(const float* po, const float* pl, int rows, int n_splits, void* o, float* lse,
+                                    cudaStream_t st) {
+  const size_t sm = size_t(n_splits) * (sizeof(float) + sizeof(int));  // weights + live split list
+  if (sm > 48 * 1024 &&
+      ensure_dyn_smem(reinterpret_cast<const void*>(decode_combine_kernel<D>), int(sm)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  decode_combine_kernel<D><<<dim3(rows), CombCfg<D>::NT, sm, st>>>(po, pl, rows, n_splits,
+                                                                   reinterpret_cast<__nv_bfloat16*>(o), lse);
+  return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
+}
+
 attn_status_t decode_combine_dispatch(const float* po, const float* pl, int rows, int n_splits, int d, void* o,
                                       float* lse, cudaStream_t st) {
-  const dim3 grid(rows);
-  __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(o);
-  const size_t sm = size_t(n_splits) * (sizeof(float) + sizeof(int));  // weights + live split list
-  if (sm > 200 * 1024) return ATTN_ERR_UNSUPPORTED;
+  if (!combine_fits(n_splits)) return ATTN_ERR_UNSUPPORTED;
   switch (d) {
-    case 64:
-      if (sm > 48 * 1024) cudaFuncSetAttribute(decode_combine_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm));
-      decode_combine_kernel<64><<<grid, CombCfg<64>::NT, sm, st>>>(po, pl, rows, n_splits, ob, lse);
-      break;
-    case 128:
-      if (sm > 48 * 1024) cudaFuncSetAttribute(decode_combine_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm));
-      decode_combine_kernel<128><<<grid, CombCfg<128>::NT, sm, st>>>(po, pl, rows, n_splits, ob, lse);
-      break;
-    case 256:
-      if (sm > 48 * 1024) cudaFuncSetAttribute(decode_combine_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm));
-      decode_combine_kernel<256><<<grid, CombCfg<256>::NT, sm, st>>>(po, pl, rows, n_splits, ob, lse);
-      break;
+    case 32: return launch_combine<32>(po, pl, rows, n_splits, o, lse, st);
+    case 64: return launch_combine<64>(po, pl, rows, n_splits, o, lse, st);
+    case 128: return launch_combine<128>(po, pl, rows, n_splits, o, lse, st);
+    case 256: return launch_combine<256>(po, pl, rows, n_splits, o, lse, st);
     default: return ATTN_ERR_UNSUPPORTED;
   }
-  return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
 }
 
 }  // namespace attn

@@ -21,7 +21,6 @@ static_assert(ATTN_DECODE_STATIC_SCRATCH_BYTES % 256 == 0, "scratch size");
 // for its device address once per device.
 static __device__ __align__(256) unsigned char g_decode_scratch[ATTN_DECODE_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 128;
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
@@ -60,9 +59,12 @@ extern "C" attn_status_t attn_decode_splitkv_static(const void* q, const void* k
     return ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
   const int G = Hq / Hkv;
-  if ((d != 64 && d != 128 && d != 256) || (G != 1 && G != 2 && G != 4 && G != 8)) return ATTN_ERR_UNSUPPORTED;
-  if (Hkv > 65535 || B > 65535) return ATTN_ERR_UNSUPPORTED;
+  if ((d != 32 && d != 64 && d != 128 && d != 256) || (G != 1 && G != 2 && G != 4 && G != 8))
+    return ATTN_ERR_UNSUPPORTED;
   if (chunk == 0) chunk = decode_default_chunk(B, Hkv, Nkv_cap);
+  // every size check comes before the split kernel is enqueued, so a refused call leaves nothing behind
+  if (Hkv > 65535 || B > 65535 || !combine_fits((Nkv_cap + (long long)chunk - 1) / chunk))
+    return ATTN_ERR_UNSUPPORTED;
   // The partials must fit the fixed array; a larger chunk makes them smaller.
   if (decode_workspace(B, Hq, d, Nkv_cap, chunk) > size_t(ATTN_DECODE_STATIC_SCRATCH_BYTES))
     return ATTN_ERR_WORKSPACE;

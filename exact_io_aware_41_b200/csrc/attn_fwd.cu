@@ -796,13 +796,8 @@ static attn_status_t launch_fwd(const void* q, const void* k, const void* v, voi
       !encode_tile_map(&tmV, v, D, Hkv, Nkv, B, C::CHUNK, C::BN, swz))
     return ATTN_ERR_CUDA;
 
-  static bool attr_set = false;  // per template instance; the attribute is per-function and sticky
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-        cudaSuccess)
-      return ATTN_ERR_CUDA;
-    attr_set = true;
-  }
+  if (ensure_dyn_smem(reinterpret_cast<const void*>(attn_fwd_kernel<D>), C::SMEM_BYTES) != cudaSuccess)
+    return ATTN_ERR_CUDA;
   FwdArgs a;
   a.o = o;
   a.lse = lse;

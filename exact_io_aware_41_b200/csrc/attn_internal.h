@@ -32,15 +32,32 @@ struct FwdArgs {
   unsigned long long timeout_ns;
 };
 
-// A 4-d TMA map over a token-major bf16 tensor [outer, rows, heads, d] (d innermost), with a box
-// of `box_cols` elements of d x 1 head x `box_rows` tokens x 1 batch. Returns false on failure.
 bool is_aligned16(const void* p);
 
-// Streaming multiprocessors of the current device (-1 on error).
+// Devices the per-device host tables cover (device ordinals 0 .. kMaxDevices-1).
+constexpr int kMaxDevices = 128;
+
+// Streaming multiprocessors of the current device (-1 on error), looked up once per device.
 int sm_count();
 
+// A 4-d TMA map over a token-major bf16 tensor [outer, rows, heads, d] (d innermost), with a box
+// of `box_cols` elements of d x 1 head x `box_rows` tokens x 1 batch; swizzle_bytes is 128, 64 or 0
+// (none). Maps are cached per (pointer, shape, box, swizzle): a map holds only the address and the
+// geometry, so a cached copy is valid wherever the same key comes back. Returns false on failure.
 bool encode_tile_map(CUtensorMap* map, const void* base, int d, int heads, int rows, int outer, int box_cols,
                      int box_rows, unsigned swizzle_bytes);
+
+// Opts `func` into `bytes` of dynamic shared memory on the current device. The attribute belongs to
+// the function on one device, so it is set once per (function, device) and again only when a
+// larger size is asked for; safe to call from several host threads.
+cudaError_t ensure_dyn_smem(const void* func, int bytes);
+
+// Largest dynamic shared memory the decode combine kernel takes (its per-split weights and live
+// split list, 8 bytes per split).
+constexpr size_t kCombineSmemMax = 200 * 1024;
+inline bool combine_fits(long long n_splits) {
+  return n_splits >= 1 && size_t(n_splits) * (sizeof(float) + sizeof(int)) <= kCombineSmemMax;
+}
 
 attn_status_t fwd_dispatch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                            int Hkv, int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream);

@@ -58,6 +58,12 @@ typedef enum {
  *   B, Hq, Hkv, Nq, Nkv >= 1; d in {32, 64, 128, 256}; scale > 0 and finite (1/sqrt(d) usually);
  *   causal 0 or 1.
  * Returns ATTN_OK once the kernel is enqueued.
+ *
+ * Concurrency: the persistent kernel hands out its work from one of 256 claim counters in device
+ * memory, assigned to launches round robin and returned to zero by each launch's last CTA. Launches
+ * on one stream never overlap, and launches on different streams are safe as long as fewer than
+ * 256 later prefill launches on that device start before an earlier one finishes (a launch held
+ * back behind a cross-stream wait while 256 others run past it would share a counter).
  */
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                        int Hkv, int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream);
@@ -84,9 +90,12 @@ int attn_decode_default_chunk(int B, int Hkv, int Nkv_cap);
  *   kv_lens          int32 [B] in device memory, each in [0, Nkv_cap] (out-of-range values are
  *                    clamped and flagged in the device error word)
  *   o                [B, Hq, d] bf16, written;  lse [B, Hq] fp32, written (-inf when kv_lens[b] = 0)
- *   d in {64, 128, 256}; Hq / Hkv in {1, 2, 4, 8}; chunk = tokens per split (multiple of 64) or 0.
+ *   d in {32, 64, 128, 256}; Hq / Hkv in {1, 2, 4, 8}; chunk = tokens per split (multiple of 64)
+ *                    or 0 (automatic: about eight splits per SM of the current device).
  *   workspace        caller-owned device memory of at least attn_decode_workspace_bytes(...) bytes;
  *                    fully overwritten before it is read, so it needs no initialisation.
+ * Sizes the kernels cannot take (B or Hkv above 65535, more than 25600 splits per row) return
+ * ATTN_ERR_UNSUPPORTED before either kernel is enqueued.
  */
 attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
                                   const int32_t* kv_lens, int Nkv_cap, void* o, float* lse, int B, int Hq,
@@ -95,7 +104,11 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
 
 /*
  * Size of the fixed device array that attn_decode_splitkv_static keeps its partials in (48 MiB).
- * The array belongs to the loaded library: every GPU that loads it holds these bytes until exit.
+ * The array belongs to the library's device code: it is committed on a GPU when that code is first
+ * loaded there (with CUDA's default lazy loading, the first call of any library entry point that
+ * launches a kernel, or the address look-up below), and held until the process exits. Under memory
+ * pressure that first load can fail and surfaces as ATTN_ERR_CUDA, so make one warm-up call at
+ * start-up.
  */
 #define ATTN_DECODE_STATIC_SCRATCH_BYTES (48u << 20)
 
@@ -112,7 +125,8 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
  *  - Sizes whose partials (see attn_decode_workspace_bytes) exceed that array are rejected with
  *    ATTN_ERR_WORKSPACE before anything is enqueued; a larger chunk makes the partials smaller.
  *  - The first call on each device looks up the array's device address on the current device
- *    (cudaGetSymbolAddress) and caches it; make that first call before any stream capture.
+ *    (cudaGetSymbolAddress), which also loads the library's device code there and commits the
+ *    array, and caches it; make that first call at start-up, before any stream capture.
  *  - Every call shares the one array and it keeps the last call's partials. Calls that overlap on
  *    the GPU (on different streams, or from different host threads without ordering) race on it.
  */
@@ -129,7 +143,7 @@ attn_status_t attn_decode_splitkv_static(const void* q, const void* k_cache, con
  *   part_o   fp32 [rows, n_splits, d] (each o_s already normalised by its own sum)
  *   part_lse fp32 [rows, n_splits]
  *   o        bf16 [rows, d], written;  lse fp32 [rows], written
- *   rows >= 1, n_splits >= 1, d in {64, 128, 256}.
+ *   rows >= 1, 1 <= n_splits <= 25600, d in {32, 64, 128, 256}.
  */
 attn_status_t attn_decode_combine(const float* part_o, const float* part_lse, int rows, int n_splits, int d,
                                   void* o, float* lse, cudaStream_t stream);

@@ -1,6 +1,9 @@
 """Helpers shared by the GPU parity tests: seeded inputs on both sides, oracle rows, tolerances."""
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 import oracle
@@ -48,45 +51,35 @@ def draw_prefill(seed, B, Hq, Hkv, Nq, Nkv, d):
             synth.normal_bf16(seed, synth.STREAM_V, (B, Nkv, Hkv, d)))
 
 
-def kv_slice_bits(seed, stream, shape, b, g, n):
-    """bf16 bits of tensor[b, :n, g, :] of a [B, N, H, d] stream, drawn on its own."""
-    _, N, H, d = shape
-    t = np.arange(n, dtype=np.int64)[:, None]
-    e = np.arange(d, dtype=np.int64)[None, :]
-    flat = ((b * N + t) * H + g) * d + e
-    return synth.normal_bf16_at(seed, stream, flat.reshape(-1)).reshape(n, d)
+def device_bits(t) -> np.ndarray:
+    """The exact bf16 bit patterns of a device tensor, copied to the host (uint16, same shape)."""
+    import torch
+
+    return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
-def q_row_bits(seed, shape, b, i, h):
-    _, N, H, d = shape
-    flat = ((b * N + i) * H + h) * d + np.arange(d, dtype=np.int64)
-    return synth.normal_bf16_at(seed, synth.STREAM_Q, flat)
+def oracle_whole_prefill(qbits, kbits, vbits, scale, causal, workers=None):
+    """The oracle's O [B, Nq, Hq, d] and LSE [B, Nq, Hq] over the whole output, one (b, h) head per
+    task: each task widens its head's bf16 bits and calls oracle.attention on that head alone. Tasks
+    run on a thread pool (the BLAS products and numpy's elementwise passes release the GIL) with one
+    BLAS thread each."""
+    from threadpoolctl import threadpool_limits
 
+    B, Nq, Hq, d = qbits.shape
+    Hkv = kbits.shape[2]
+    O = np.empty((B, Nq, Hq, d))
+    L = np.empty((B, Nq, Hq))
+    f = synth.bf16_bits_to_f64
 
-def sample_rows(rng, B, Nq, Hq, n, causal):
-    """A fixed set of (b, i, h) triples: corners, tile edges, and random rows."""
-    picks = {(0, 0, 0), (B - 1, Nq - 1, Hq - 1), (0, Nq - 1, 0), (B - 1, 0, Hq - 1)}
-    for i in (127, 128, 255, 256, 383, 384, Nq // 2):
-        if i < Nq:
-            picks.add((int(rng.integers(B)), i, int(rng.integers(Hq))))
-    while len(picks) < n:
-        picks.add((int(rng.integers(B)), int(rng.integers(Nq)), int(rng.integers(Hq))))
-    return sorted(picks)
+    def head(bh):
+        b, h = divmod(bh, Hq)
+        g = oracle.kv_head(h, Hq, Hkv)
+        o, lse = oracle.attention(f(qbits[b:b + 1, :, h:h + 1]), f(kbits[b:b + 1, :, g:g + 1]),
+                                  f(vbits[b:b + 1, :, g:g + 1]), scale, causal)
+        O[b, :, h] = o[0, :, 0]
+        L[b, :, h] = lse[0, 0]
 
-
-def oracle_rows_prefill(w, picks):
-    """Oracle O rows and LSE for the sampled (b, i, h) of a prefill workload drawn from its seed."""
-    qshape = (w.B, w.Nq, w.Hq, w.d)
-    kshape = (w.B, w.Nkv, w.Hkv, w.d)
-    cache = {}
-    outs = []
-    for (b, i, h) in picks:
-        g = oracle.kv_head(h, w.Hq, w.Hkv)
-        if (b, g) not in cache:
-            cache[(b, g)] = (synth.bf16_bits_to_f64(kv_slice_bits(w.seed, synth.STREAM_K, kshape, b, g, w.Nkv)),
-                             synth.bf16_bits_to_f64(kv_slice_bits(w.seed, synth.STREAM_V, kshape, b, g, w.Nkv)))
-        K, V = cache[(b, g)]
-        keys = oracle.visible_keys(i, w.Nq, w.Nkv, w.causal)
-        q = synth.bf16_bits_to_f64(q_row_bits(w.seed, qshape, b, i, h))
-        outs.append(oracle.attention_row(q, K[keys], V[keys], w.scale))
-    return np.array([o for o, _ in outs]), np.array([l for _, l in outs])
+    n = workers or max(1, min(8, os.cpu_count() or 1))
+    with threadpool_limits(limits=1, user_api="blas"), ThreadPoolExecutor(n) as ex:
+        list(ex.map(head, range(B * Hq)))
+    return O, L

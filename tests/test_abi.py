@@ -94,13 +94,32 @@ def test_argument_errors_are_reported_before_any_launch(raw):
     assert lib.attn_decode_splitkv(*args, 100, p, 1 << 30, None) == pkg.ATTN_ERR_INVALID_ARG
     assert lib.attn_decode_splitkv(p, p, p, p, 1024, p, p, 2, 6, 2, 128, 0.1, 64, p, 1 << 30, None) == \
         pkg.ATTN_ERR_UNSUPPORTED
-    assert lib.attn_decode_splitkv(p, p, p, p, 1024, p, p, 2, 8, 2, 32, 0.1, 64, p, 1 << 30, None) == \
+    assert lib.attn_decode_splitkv(p, p, p, p, 1024, p, p, 2, 8, 2, 48, 0.1, 64, p, 1 << 30, None) == \
         pkg.ATTN_ERR_UNSUPPORTED
     assert lib.attn_decode_splitkv(*args, 64, p, 16, None) == pkg.ATTN_ERR_WORKSPACE
     assert lib.attn_decode_splitkv(*args, 64, 0, 1 << 30, None) == pkg.ATTN_ERR_WORKSPACE
     assert lib.attn_decode_combine(p, p, 0, 4, 128, p, p, None) == pkg.ATTN_ERR_INVALID_ARG
     assert lib.attn_decode_combine(p, p, 4, 4, 96, p, p, None) == pkg.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_decode_combine(p, p, 4, 25601, 128, p, p, None) == pkg.ATTN_ERR_UNSUPPORTED
     assert lib.attn_selftest_bounded_wait(0, None) == pkg.ATTN_ERR_INVALID_ARG
     assert lib.attn_selftest_exp2_poly(None, p, 4, None) == pkg.ATTN_ERR_INVALID_ARG
     assert lib.attn_selftest_exp2_poly(p, p, 0, None) == pkg.ATTN_ERR_INVALID_ARG
     assert lib.attn_selftest_exp2_poly(p + 2, p, 4, None) == pkg.ATTN_ERR_INVALID_ARG
+
+
+def test_decode_sizes_the_combine_cannot_take_are_refused_before_any_launch(raw):
+    """More than 25600 splits per row (the combine kernel's shared-memory limit) is refused by both
+    decode entry points before the split kernel is enqueued: no CUDA call is reached here, on a
+    host without a GPU."""
+    import exact_io_aware_41_b200 as pkg
+
+    lib = pkg.lib_handle()
+    p = 1 << 20
+    cap = 64 * 25601  # chunk 64: 25601 splits
+    assert lib.attn_decode_splitkv(p, p, p, p, cap, p, p, 1, 1, 1, 32, 0.1, 64, p, 1 << 40, None) == \
+        pkg.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_decode_splitkv_static(p, p, p, p, cap, p, p, 1, 1, 1, 32, 0.1, 64, None) == \
+        pkg.ATTN_ERR_UNSUPPORTED
+    # one split fewer passes the check and reaches the workspace check (too small here)
+    assert lib.attn_decode_splitkv(p, p, p, p, cap - 64, p, p, 1, 1, 1, 32, 0.1, 64, p, 16, None) == \
+        pkg.ATTN_ERR_WORKSPACE

@@ -57,11 +57,21 @@ def test_ncu_traffic_is_keyed_to_the_kernel_source():
 
 
 def test_ncu_traffic_stale_key_reports_nothing(monkeypatch):
-    path, digest, nbytes = bench.NCU_TRAFFIC["decode"]
-    monkeypatch.setitem(bench.NCU_TRAFFIC, "decode", (path, "0" * 64, nbytes))
-    assert bench.ncu_traffic("decode") is None
-    monkeypatch.setitem(bench.NCU_TRAFFIC, "decode", ("no/such/file.cu", digest, nbytes))
-    assert bench.ncu_traffic("decode") is None
+    key = bench.synth.DECODE.name
+    path, digest, nbytes = bench.NCU_TRAFFIC[key]
+    monkeypatch.setitem(bench.NCU_TRAFFIC, key, (path, "0" * 64, nbytes))
+    assert bench.ncu_traffic(key) is None
+    monkeypatch.setitem(bench.NCU_TRAFFIC, key, ("no/such/file.cu", digest, nbytes))
+    assert bench.ncu_traffic(key) is None
+    assert bench.ncu_traffic("a workload nobody measured") is None
+
+
+def test_prefill_algorithmic_bytes():
+    w = bench.synth.LONG_8K
+    # q, k, v, O: 2 * 8192 * 16 * 128 * 2 bytes each; LSE 2 * 16 * 8192 * 4 bytes
+    assert bench.prefill_bytes(w) == 4 * 67108864 + 1048576
+    g = bench.synth.LONG_8K_GQA
+    assert bench.prefill_bytes(g) == 2 * 134217728 + 2 * 33554432 + 2097152
 
 
 def test_max_over_ranks_single_process():

@@ -1,5 +1,5 @@
 """Split-KV decode parity: CUDA path (split kernel + combine, through the C ABI) against the fp64
-oracle, on small shapes compared whole and on the full decode workload compared on sampled rows."""
+oracle, on small shapes and on every row of the full decode workload."""
 import math
 
 import numpy as np
@@ -7,7 +7,7 @@ import pytest
 
 import oracle
 import synth
-from parity import assert_parity, bf16_tensor_to_f64, kv_slice_bits, to_torch_bf16
+from parity import assert_parity, bf16_tensor_to_f64, device_bits, to_torch_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -30,7 +30,7 @@ def _decode_small(lib, seed, B, Hq, Hkv, d, cap, lens, chunk):
                   f"decode B{B} Hq{Hq} Hkv{Hkv} d{d} cap{cap} chunk{chunk}")
 
 
-@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("d", [32, 64, 128, 256])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_decode_every_head_dim_and_group(lib, d, G):
     # lengths: full cache, one token, empty, and ragged values across several 64-token splits
@@ -79,7 +79,9 @@ def test_combine_entry_point_matches_the_merge_identity(lib):
     assert_parity(bf16_tensor_to_f64(o), lse.cpu().numpy().astype(np.float64), O_ref, L_ref, "combine")
 
 
-def test_full_decode_workload_sampled(lib):
+def test_full_decode_workload_every_row(lib):
+    """The full decode workload (eight sequences of 1k-128k tokens, GQA 32/8), all 256 (b, hq) rows
+    against oracle.decode, fed the exact bits the kernels read (copied back one sequence at a time)."""
     import torch
 
     w = synth.DECODE
@@ -93,24 +95,43 @@ def test_full_decode_workload_sampled(lib):
     o, lse = lib.attn_decode_splitkv(q, kc, vc, lens_t, scale=w.scale)
     torch.cuda.synchronize()
     assert lib.attn_get_last_error() == lib.ATTN_OK
-    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
-
-    qh = synth.bf16_bits_to_f64(q.cpu().view(torch.int16).numpy().view(np.uint16))
-    qbits = synth.normal_bf16(w.seed, synth.STREAM_Q, (w.B, w.Hq, w.d))
-    assert np.array_equal(synth.bf16_bits_to_f64(qbits), qh)
-    G = w.Hq // w.Hkv
-    # the shortest and longest sequences and one in between, every query head of one kv head each
-    order = np.argsort(lens)
-    picks = [(int(order[0]), 0), (int(order[-1]), w.Hkv - 1), (int(order[len(order) // 2]), 3)]
-    for b, g in picks:
+    qh = synth.bf16_bits_to_f64(device_bits(q))
+    O_ref = np.zeros((w.B, w.Hq, w.d))
+    L_ref = np.zeros((w.B, w.Hq))
+    for b in range(w.B):
         L = int(lens[b])
-        kbits = kv_slice_bits(w.seed, synth.STREAM_K, shape, b, g, L)
-        assert np.array_equal(kc[b, :64, g].cpu().view(torch.int16).numpy().view(np.uint16), kbits[:64])
-        K = synth.bf16_bits_to_f64(kbits)
-        V = synth.bf16_bits_to_f64(kv_slice_bits(w.seed, synth.STREAM_V, shape, b, g, L))
-        rows = [oracle.attention_row(qh[b, h], K, V, w.scale) for h in range(g * G, (g + 1) * G)]
-        O_ref = np.array([r[0] for r in rows])
-        L_ref = np.array([r[1] for r in rows])
-        assert_parity(bf16_tensor_to_f64(o[b, g * G:(g + 1) * G]),
-                      lse[b, g * G:(g + 1) * G].cpu().numpy().astype(np.float64), O_ref, L_ref,
-                      f"decode b={b} L={L} g={g}")
+        kb = synth.bf16_bits_to_f64(device_bits(kc[b:b + 1, :L]))
+        vb = synth.bf16_bits_to_f64(device_bits(vc[b:b + 1, :L]))
+        O_ref[b:b + 1], L_ref[b:b + 1] = oracle.decode(qh[b:b + 1], kb, vb, np.array([L]), w.scale)
+        del kb, vb
+    assert_parity(bf16_tensor_to_f64(o), lse.cpu().numpy().astype(np.float64), O_ref, L_ref,
+                  "full decode workload, all rows")
+
+
+def test_refused_sizes_launch_nothing(lib):
+    """More splits per row than the combine kernel takes: UNSUPPORTED, and the outputs keep their
+    previous contents (nothing was launched). The buffers are sized for the requested shape, so even
+    a launch would have stayed in bounds."""
+    import ctypes
+
+    import torch
+
+    B, Hq, Hkv, d, chunk = 1, 1, 1, 32, 64
+    cap = chunk * 25601
+    kc = torch.zeros((B, cap, Hkv, d), dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros((B, Hq, d), dtype=torch.bfloat16, device="cuda")
+    lens = torch.zeros(B, dtype=torch.int32, device="cuda")
+    o = torch.full((B, Hq, d), 3.0, dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, Hq), 5.0, dtype=torch.float32, device="cuda")
+    ws = torch.empty(lib.attn_decode_workspace_bytes(B, Hq, Hkv, d, cap, chunk), dtype=torch.uint8, device="cuda")
+    st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    h = lib.lib_handle()
+    assert h.attn_decode_splitkv(q.data_ptr(), kc.data_ptr(), kc.data_ptr(), lens.data_ptr(), cap, o.data_ptr(),
+                                 lse.data_ptr(), B, Hq, Hkv, d, 0.125, chunk, ws.data_ptr(), ws.numel(),
+                                 st) == lib.ATTN_ERR_UNSUPPORTED
+    assert h.attn_decode_splitkv_static(q.data_ptr(), kc.data_ptr(), kc.data_ptr(), lens.data_ptr(), cap,
+                                        o.data_ptr(), lse.data_ptr(), B, Hq, Hkv, d, 0.125, chunk,
+                                        st) == lib.ATTN_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert torch.all(o.float() == 3.0) and torch.all(lse == 5.0)
+    assert lib.attn_get_last_error() == lib.ATTN_OK

@@ -1,7 +1,6 @@
 """Prefill parity: the CUDA path (through the C ABI) against the fp64 CPU oracle on the same seeded
-bf16 inputs. Small shapes are compared element by element over the whole output; the full-size
-workloads are compared on sampled rows the oracle computes one by one, plus properties that hold
-at any size."""
+bf16 inputs, element by element over the whole output: small shapes drawn on the host, and every
+full-size workload drawn on the device with the oracle fed the exact bits the kernel read."""
 import math
 
 import numpy as np
@@ -9,8 +8,8 @@ import pytest
 
 import oracle
 import synth
-from parity import (assert_parity, bf16_tensor_to_f64, draw_prefill, kv_slice_bits, oracle_rows_prefill,
-                    sample_rows, to_torch_bf16)
+from parity import (assert_parity, bf16_tensor_to_f64, device_bits, draw_prefill, oracle_whole_prefill,
+                    to_torch_bf16)
 
 pytestmark = pytest.mark.gpu
 
@@ -127,31 +126,22 @@ FULL = [synth.CAUSAL_2K, synth.LONG_8K, synth.LONG_8K_CAUSAL, synth.LONG_8K_GQA,
 
 
 @pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
-def test_full_size_workload_sampled_rows(lib, w):
+def test_full_size_workload_whole_output(lib, w):
+    """Every full-size workload, compared element by element over the whole O and LSE. The inputs
+    are drawn on the device (as the benchmark does), and the oracle is fed the exact bits the kernel
+    read, copied back to the host, so the comparison does not rest on the two draws agreeing."""
     import torch
 
     dev = "cuda"
     q = synth.normal_bf16_torch(w.seed, synth.STREAM_Q, (w.B, w.Nq, w.Hq, w.d), dev)
     k = synth.normal_bf16_torch(w.seed, synth.STREAM_K, (w.B, w.Nkv, w.Hkv, w.d), dev)
     v = synth.normal_bf16_torch(w.seed, synth.STREAM_V, (w.B, w.Nkv, w.Hkv, w.d), dev)
-    # the device draw is the host draw (checked on one kv row block)
-    host = kv_slice_bits(w.seed, synth.STREAM_K, tuple(k.shape), w.B - 1, w.Hkv - 1, 256)
-    assert np.array_equal(k[w.B - 1, :256, w.Hkv - 1].cpu().view(torch.int16).numpy().view(np.uint16), host)
-
     o, lse = lib.attn_fwd(q, k, v, scale=w.scale, causal=w.causal)
     torch.cuda.synchronize()
     assert lib.attn_get_last_error() == lib.ATTN_OK
-
-    # properties at full size: finite, and each O element inside the range of V over its kv head
-    assert torch.isfinite(o.float()).all()
-    assert torch.isfinite(lse).all()
-    vmax = v.float().abs().amax().item()
-    assert o.float().abs().amax().item() <= vmax * (1 + 2 ** -6)
-
-    rng = np.random.default_rng(w.seed)
-    picks = sample_rows(rng, w.B, w.Nq, w.Hq, 48, w.causal)
-    O_ref, L_ref = oracle_rows_prefill(w, picks)
-    idx = tuple(np.array(p) for p in zip(*picks))
-    o_s = bf16_tensor_to_f64(o[idx[0], idx[1], idx[2]])
-    l_s = lse[idx[0], idx[2], idx[1]].cpu().numpy().astype(np.float64)
-    assert_parity(o_s, l_s, O_ref, L_ref, w.name)
+    qb, kb, vb = device_bits(q), device_bits(k), device_bits(v)
+    og, lg = bf16_tensor_to_f64(o), lse.cpu().numpy().astype(np.float64).transpose(0, 2, 1)
+    del q, k, v, o, lse
+    torch.cuda.empty_cache()
+    O_ref, L_ref = oracle_whole_prefill(qb, kb, vb, w.scale, w.causal)
+    assert_parity(og, lg, O_ref, L_ref, w.name)

@@ -8,7 +8,7 @@ import pytest
 
 import oracle
 import synth
-from parity import assert_parity, bf16_tensor_to_f64, draw_prefill, to_torch_bf16
+from parity import assert_parity, bf16_tensor_to_f64, device_bits, draw_prefill, to_torch_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -106,7 +106,7 @@ def _decode_case(lib, seed, B, Hq, Hkv, d, cap, lens, chunk):
                   f"decode d{d} lens {lens} chunk {chunk}")
 
 
-@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("d", [32, 64, 128, 256])
 def test_decode_tails_straddling_tiles_with_nan_padding(lib, d):
     # lengths 1..130 around the 16- and 64-token tile edges; the unused cache rows are NaN
     _decode_case(lib, 5500 + d, 8, 8, 2, d, 192, [1, 15, 16, 17, 63, 65, 127, 130], 64)
@@ -126,3 +126,41 @@ def test_decode_all_lengths_zero(lib):
 
 def test_decode_full_cache_every_sequence(lib):
     _decode_case(lib, 5600, 2, 16, 2, 128, 4096, [4096, 4096], 0)
+
+
+def test_tensor_map_cache_same_pointer_many_shapes_two_streams(lib):
+    """The library caches TMA descriptors per (pointer, shape). Views of the same three buffers with
+    more distinct shapes than the cache holds, launched alternately on two streams and then again
+    in the same order (after their entries were evicted), must each give the oracle's result."""
+    import torch
+
+    n = 1 << 20
+    bufs = [synth.normal_bf16_torch(5700 + i, 0, (n,), "cuda") for i in range(3)]
+    shapes = []
+    for i in range(72):  # > 64 cache entries
+        d = (32, 64, 128, 256)[i % 4]
+        Hkv = 1 + (i // 4) % 2
+        Hq = Hkv * (1 + (i // 8) % 2)
+        N = 40 + 13 * i
+        shapes.append((Hq, Hkv, N, d, bool(i % 3 == 0)))
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    torch.cuda.synchronize()
+    for rep in range(2):
+        for i, (Hq, Hkv, N, d, causal) in enumerate(shapes):
+            q = bufs[0][:N * Hq * d].view(1, N, Hq, d)
+            k = bufs[1][:N * Hkv * d].view(1, N, Hkv, d)
+            v = bufs[2][:N * Hkv * d].view(1, N, Hkv, d)
+            st = streams[(i + rep) % 2]
+            with torch.cuda.stream(st):
+                outs.append(lib.attn_fwd(q, k, v, causal=causal, stream=st))
+    torch.cuda.synchronize()
+    assert lib.attn_get_last_error() == lib.ATTN_OK
+    for j, (o, lse) in enumerate(outs):
+        Hq, Hkv, N, d, causal = shapes[j % len(shapes)]
+        qb = device_bits(bufs[0][:N * Hq * d]).reshape(1, N, Hq, d)
+        kb = device_bits(bufs[1][:N * Hkv * d]).reshape(1, N, Hkv, d)
+        vb = device_bits(bufs[2][:N * Hkv * d]).reshape(1, N, Hkv, d)
+        O_ref, L_ref = _prefill_ref(qb, kb, vb, 1 / math.sqrt(d), causal)
+        assert_parity(bf16_tensor_to_f64(o), lse.cpu().numpy().astype(np.float64).transpose(0, 2, 1), O_ref,
+                      L_ref, f"shape {shapes[j % len(shapes)]} pass {j // len(shapes)}")

@@ -45,6 +45,17 @@ def test_golden_closed_forms():
         np.testing.assert_allclose(L[0, 0, :], exp_L, rtol=0, atol=1e-12, err_msg=c["name"])
 
 
+def test_golden_probabilities():
+    """oracle.probabilities against the hand-derived P of each golden case (a dropped or inverted
+    scale, or negated scores, change these values; a per-row constant does not, hence the LSE pins)."""
+    with open(os.path.join(HERE, "golden", "closed_form.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        P = oracle.probabilities(np.array(c["q"], dtype=np.float64), np.array(c["k"], dtype=np.float64),
+                                 c["scale"], c["causal"])
+        np.testing.assert_allclose(P, np.array(c["P"], dtype=np.float64), rtol=0, atol=1e-12, err_msg=c["name"])
+
+
 # -------------------------------------------------------------------------------------------
 # invariants and special cases
 # -------------------------------------------------------------------------------------------
@@ -172,6 +183,30 @@ def test_brute_force_tiny(Hq, Hkv, Nq, Nkv, causal):
     np.testing.assert_allclose(L[np.isfinite(L)], Lb[np.isfinite(Lb)], rtol=0, atol=1e-12)
 
 
+@pytest.mark.parametrize("Nq,Nkv,causal,qscale", [
+    (5, 7, False, 2.0), (7, 7, True, 2.0), (3, 6, True, 2.0), (6, 3, True, 2.0),
+    (5, 7, False, 600.0), (7, 7, True, 600.0),  # scores in the hundreds: exp overflows without a max shift
+])
+def test_probabilities_brute_force(Nq, Nkv, causal, qscale):
+    """P entry by entry in plain Python: exp(s_ij - m_i) / sum over visible j of exp(s_ij - m_i),
+    with m_i the row's largest visible score (the same ratio as exp(s_ij) / sum exp(s_ij))."""
+    rng = np.random.default_rng(30 + Nq + Nkv)
+    q, k = qscale * _rand(rng, Nq, 4), _rand(rng, Nkv, 4)
+    P = oracle.probabilities(q, k, 0.7, causal)
+    assert np.all(np.isfinite(P))
+    for i in range(Nq):
+        keys = [j for j in range(Nkv) if (not causal) or j <= i + Nkv - Nq]
+        s = {j: 0.7 * sum(float(q[i, t]) * float(k[j, t]) for t in range(4)) for j in keys}
+        if not s:  # a row that sees no key is all zero
+            assert np.all(P[i] == 0.0)
+            continue
+        m = max(s.values())
+        z = sum(math.exp(x - m) for x in s.values())
+        for j in range(Nkv):
+            want = math.exp(s[j] - m) / z if j in s else 0.0
+            assert abs(P[i, j] - want) < 1e-12, (i, j)
+
+
 # -------------------------------------------------------------------------------------------
 # an independent library routine
 # -------------------------------------------------------------------------------------------
@@ -221,10 +256,15 @@ def test_linear_in_v_and_key_permutation_invariant():
     O3, L3 = oracle.attention(q, k[:, perm], v[:, perm], 0.8, False)
     np.testing.assert_allclose(O3, O, rtol=0, atol=1e-12)
     np.testing.assert_allclose(L3, L, rtol=0, atol=1e-12)
-    # shifting every score of a row by the same amount moves LSE and leaves O alone
-    shift = np.zeros_like(k)
-    O4, L4 = oracle.attention(q, k + shift, v, 0.8, False)
-    assert np.array_equal(O4, O)
+    # shifting every score of row i by the same amount a_i moves LSE[i] by a_i and leaves O alone:
+    # append a coordinate a_i / scale to q_i and 1 to every key
+    a = rng.uniform(-3.0, 3.0, size=(1, 5, 2))
+    q5 = np.concatenate([q, (a / 0.8)[..., None]], axis=-1)
+    k5 = np.concatenate([k, np.ones(k.shape[:-1] + (1,))], axis=-1)
+    v5 = np.concatenate([v, np.zeros(v.shape[:-1] + (1,))], axis=-1)
+    O4, L4 = oracle.attention(q5, k5, v5, 0.8, False)
+    np.testing.assert_allclose(O4[..., :-1], O, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L4, L + a.transpose(0, 2, 1), rtol=0, atol=1e-12)
 
 
 def test_scale_enters_as_a_factor_on_scores():

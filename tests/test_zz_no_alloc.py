@@ -3,9 +3,9 @@
 Some callers cannot hand the library a workspace: a plugin inside a host runtime that owns all
 device memory, or a serving loop that must not call cudaMalloc. For them the library keeps the
 split partials in one fixed device array. These checks call that entry point through the C ABI and
-compare it with the workspace entry point on the same inputs, twice in a row with different inputs
-(the array keeps the previous call's partials, which must not leak into the next result). The file
-is named so pytest collects it last.
+compare it with the workspace entry point and with the fp64 oracle on the same inputs, twice in a
+row with different inputs (the array keeps the previous call's partials, which must not leak into
+the next result). The file is named so pytest collects it last.
 """
 import ctypes
 import math
@@ -13,8 +13,9 @@ import math
 import numpy as np
 import pytest
 
+import oracle
 import synth
-from parity import assert_parity, bf16_tensor_to_f64
+from parity import assert_parity, bf16_tensor_to_f64, device_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -47,6 +48,11 @@ def test_static_scratch_decode_matches_workspace_decode_twice(lib):
         assert lib.attn_get_last_error() == lib.ATTN_OK
         assert_parity(bf16_tensor_to_f64(o), lse.cpu().numpy().astype(np.float64),
                       bf16_tensor_to_f64(o_ref), l_ref.cpu().numpy().astype(np.float64), f"static decode call {call}")
+        # and against the fp64 oracle on the exact inputs
+        O_or, L_or = oracle.decode(synth.bf16_bits_to_f64(device_bits(q)), synth.bf16_bits_to_f64(device_bits(kc)),
+                                   synth.bf16_bits_to_f64(device_bits(vc)), np.array(lens), 1.0 / math.sqrt(d))
+        assert_parity(bf16_tensor_to_f64(o), lse.cpu().numpy().astype(np.float64), O_or, L_or,
+                      f"static decode call {call} vs oracle")
 
 
 def test_static_scratch_decode_binding_and_size_limit(lib):
