@@ -46,11 +46,29 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 # that file changes, the figure is stale and the bench line reports null until it is measured again.
 PREFILL_SRC = "exact_io_aware_41_b200/csrc/attn_fwd.cu"
 DECODE_SRC = "exact_io_aware_41_b200/csrc/attn_decode.cu"
+PREFILL_SHA = "ab469009540e1a218be3af0398ce49023e016c49ac7226da759dd84960e98ae8"  # sha256 of PREFILL_SRC when the prefill figures were taken
 NCU_TRAFFIC = {
-    # decode_split_tc_kernel<128,4> (2123.74 MB read + 7.08 MB written) + decode_combine_kernel<128>
+    # attn_fwd_kernel: 337.62 MB read + 49.63 MB written
+    synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 387_250_944.0),
+    # attn_fwd_kernel: 122.96 MB read + 9.71 MB written
+    synth.CAUSAL_2K.name: (PREFILL_SRC, PREFILL_SHA, 132_674_304.0),
+    # attn_fwd_kernel: 210.23 MB read + 47.78 MB written
+    synth.LONG_8K_CAUSAL.name: (PREFILL_SRC, PREFILL_SHA, 258_014_208.0),
+    # attn_fwd_kernel: 323.59 MB read + 101.11 MB written
+    synth.LONG_8K_GQA.name: (PREFILL_SRC, PREFILL_SHA, 424_704_000.0),
+    # attn_fwd_kernel: 369.60 MB read + 96.79 MB written
+    synth.LONG_8K_GQA_CAUSAL.name: (PREFILL_SRC, PREFILL_SHA, 466_393_344.0),
+    # attn_fwd_kernel: 50.45 MB read + 1.51 MB written
+    synth.SWEEP[0].name: (PREFILL_SRC, PREFILL_SHA, 51_952_128.0),
+    # attn_fwd_kernel: 116.12 MB read + 22.65 MB written
+    synth.SWEEP[1].name: (PREFILL_SRC, PREFILL_SHA, 138_769_664.0),
+    # attn_fwd_kernel: 330.37 MB read + 49.33 MB written
+    synth.SWEEP[2].name: (PREFILL_SRC, PREFILL_SHA, 379_698_432.0),
+    # attn_fwd_kernel: 689.65 MB read + 117.05 MB written
+    synth.SWEEP[3].name: (PREFILL_SRC, PREFILL_SHA, 806_694_400.0),
+    # decode_split_tc_kernel<128,4> (2123.81 MB read + 7.59 MB written) + decode_combine_kernel<128>
     # (4.29 MB read) on the full decode workload
-    synth.DECODE.name: (DECODE_SRC, "8f7ae30438212f2aa0baa6b8c3896abe248dbfb72e17985d9f09ab0e1293ef52",
-                        2_135_109_632.0),
+    synth.DECODE.name: (DECODE_SRC, "eaf4990882bbcba5d723de8f5b505ab0c1520f88553cb35fa7ee6758aa501c3a", 2_135_693_824.0),
 }
 
 

@@ -47,14 +47,23 @@ constexpr double kL2OneGroupBytes = ATTN_L2_ONE_GROUP_MB * 1.0e6;
 // Running-max slack before O is rescaled, in log2 units: P entries stay <= 2^TAU.
 constexpr float kRescaleTau = 8.0f;
 
-// Columns (per 128 keys) whose exponential is evaluated on the FMA pipe instead of the exp unit,
-// in tiles without masked keys (the exp unit and the tensor cores need about the same number of
-// cycles per tile at d = 128, so moving part of the exponentials frees the bottleneck).
-#ifndef ATTN_EMU_COLS
-#define ATTN_EMU_COLS 0
+// Columns (per 128 keys) whose exponential is evaluated on the FMA pipe instead of the exp unit, in
+// tiles without masked keys, per head dim. Every tile needs BM x BN exponentials whatever d is, so
+// the exp unit bounds the softmax; moving part of them to the FMA pipe relieves it only when the
+// FMA pipe has room and enough independent pairs are in flight. Measured on B200 it did not pay at
+// any head dim, so the product builds use none; the variant is built and checked by the tests.
+#ifndef ATTN_EMU_COLS_D32
+#define ATTN_EMU_COLS_D32 0
 #endif
-constexpr int kEmuCols = ATTN_EMU_COLS;
-static_assert(kEmuCols % 8 == 0 && kEmuCols >= 0 && kEmuCols <= 128, "emulated column count");
+#ifndef ATTN_EMU_COLS_D64
+#define ATTN_EMU_COLS_D64 0
+#endif
+#ifndef ATTN_EMU_COLS_D128
+#define ATTN_EMU_COLS_D128 0
+#endif
+#ifndef ATTN_EMU_COLS_D256
+#define ATTN_EMU_COLS_D256 0
+#endif
 
 template <int D>
 struct FwdCfg {
@@ -77,6 +86,15 @@ struct FwdCfg {
   static constexpr int STAGES = (D == 256) ? 5 : (KV_TILE_BYTES >= 32768) ? 4 : 8;
   static constexpr int NSMWG = (NQT == 2) ? 2 : 1;      // softmax warpgroups
   static constexpr int THREADS = 128 * (1 + NSMWG);
+  // register split (setmaxnreg) with two softmax warpgroups: control warpgroup, softmax warpgroups;
+  // the sum must fit in the launch allocation (THREADS x the kernel's register count, checked on the
+  // host before the first launch)
+  static constexpr bool SPLIT_REGS = (NQT == 2);
+  static constexpr int CTRL_REGS = 104;
+  static constexpr int SM_REGS = 192;
+  static constexpr int EMU_COLS = D == 32 ? ATTN_EMU_COLS_D32 : D == 64 ? ATTN_EMU_COLS_D64
+                                  : D == 128 ? ATTN_EMU_COLS_D128 : ATTN_EMU_COLS_D256;
+  static_assert(EMU_COLS % 8 == 0 && EMU_COLS >= 0 && EMU_COLS <= 128, "emulated column count");
   static constexpr int HALF_PAIRS = BN / 4;             // bf16 pairs (TMEM columns) of P per half tile
   static constexpr int PV_KH = BN / 32;                 // PV k-steps (16 keys) per half tile
   // TMEM columns (fp32 each): two S slots, then one O accumulator per query tile.
@@ -234,7 +252,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   // With two softmax warpgroups the 128 control threads give registers to the 256 softmax threads:
   // 128 * 104 + 256 * 192 = 62464 <= 384 * 168 (the launch allocation). Each role changes its budget
   // at the top of its own branch so the new limit covers all of that role's code.
-  constexpr bool kSplitRegs = (C::NQT == 2);
+  constexpr bool kSplitRegs = C::SPLIT_REGS;
 
   // ---- MMA issue helpers ------------------------------------------------------------------------
   constexpr uint32_t idesc_qk = idesc_bf16_f32(128, C::BN, 0, 0);
@@ -299,7 +317,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 
   if (warp == 0) {
     // ================================ TMA producer ================================
-    if (kSplitRegs) regs_dec<104>();
+    if (kSplitRegs) regs_dec<C::CTRL_REGS>();
     if (lane == 0) {
       bool ok = true;
       int pos = 0;  // next ring position
@@ -362,7 +380,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ================================ MMA issuer ================================
-    if (kSplitRegs) regs_dec<104>();
+    if (kSplitRegs) regs_dec<C::CTRL_REGS>();
     if (lane == 0) {
       // K/V tiles and Q arrive by TMA (complete_tx on the mbarrier): the MMAs may read them once the
       // barrier phase is observed. P is written to TMEM by the softmax threads' tcgen05.st, so
@@ -527,10 +545,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     }
     __syncwarp();
   } else if (warp < 4) {
-    if (kSplitRegs) regs_dec<104>();
+    if (kSplitRegs) regs_dec<C::CTRL_REGS>();
   } else {
     // ================================ softmax warpgroups ================================
-    if (kSplitRegs) regs_inc<192>();
+    if (kSplitRegs) regs_inc<C::SM_REGS>();
     const int wg = (warp - 4) >> 2;
     const int wq = warp & 3;             // warp within its warpgroup: TMEM lanes 32*wq .. 32*wq+31
     const int row = wq * 32 + lane;      // query row within the tile = TMEM lane
@@ -670,14 +688,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         // P = 2^(c*s - c*m_ref) as bf16 over the first BN/2 columns of the slot (two per 32-bit
         // column; the S values it replaces are already in registers). Pairs go through the packed
         // FMA pipe; the exponential uses the exp unit (MUFU.EX2) or, for the last kEmuCols columns
-        // of tiles without masked keys, the FMA-pipe polynomial.
+        // of tiles without masked keys, the FMA-pipe polynomial (EMU_COLS).
         const float mc = (m_ref == -INFINITY) ? 0.f : m_ref * c;
         const float2 c2 = make_float2(c, c);
         const float2 nmc2 = make_float2(-mc, -mc);
         float2 acc4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                           make_float2(0.f, 0.f)};
-        constexpr int EMU_FROM = (C::BN - kEmuCols * C::BN / 128) / 2;  // first emulated pair
-        const bool emu = kEmuCols > 0 && !need_mask;
+        constexpr int EMU_FROM = (C::BN - C::EMU_COLS * C::BN / 128) / 2;  // first emulated pair
+        const bool emu = C::EMU_COLS > 0 && !need_mask;
         if (!wait_prev_pv()) {  // the P buffer is free again
           ok = false;
           break;
@@ -798,6 +816,21 @@ static attn_status_t launch_fwd(const void* q, const void* k, const void* v, voi
 
   if (ensure_dyn_smem(reinterpret_cast<const void*>(attn_fwd_kernel<D>), C::SMEM_BYTES) != cudaSuccess)
     return ATTN_ERR_CUDA;
+  // setmaxnreg.inc waits until the registers it asks for are free in the CTA's launch allocation,
+  // so a split whose total exceeds that allocation would never proceed: refuse to launch it.
+  if (C::SPLIT_REGS) {
+    static std::atomic<int> regs_ok{0};  // 0 unknown, 1 fits, 2 does not (same binary on every device)
+    int st = regs_ok.load(std::memory_order_relaxed);
+    if (st == 0) {
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D>) != cudaSuccess) return ATTN_ERR_CUDA;
+      const long long pool = (long long)fa.numRegs * C::THREADS;
+      const long long need = 128LL * C::CTRL_REGS + 128LL * C::NSMWG * C::SM_REGS;
+      st = pool >= need ? 1 : 2;
+      regs_ok.store(st, std::memory_order_relaxed);
+    }
+    if (st != 1) return ATTN_ERR_UNSUPPORTED;
+  }
   FwdArgs a;
   a.o = o;
   a.lse = lse;
