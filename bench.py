@@ -349,6 +349,8 @@ def run_ours(args, world, rank, local, dist):
         for w in GATES:
             gates[w.name] = time_prefill(lib, w, dev, stream, peaks)
             torch.cuda.empty_cache()
+        gates["fp8 " + P.name] = time_prefill_fp8(lib, P, dev, stream, peaks)
+        torch.cuda.empty_cache()
 
     # ---- end to end through the public API with pinned host buffers
     e2e = e2e_prefill(lib, P, q, k, v, stream, max(3, min(K, 50)))
@@ -391,7 +393,7 @@ def run_ours(args, world, rank, local, dist):
                   "prefill inputs; gates flush L2 (256 MiB write) before every launch",
         },
         "frac_of_nominal_bf16": pf_tflops_1 / NOMINAL_BF16_TFLOPS,
-        "roofline": {"bound": "tensor", "kernel": lib.kernel_name(0).replace("<D>", "<128>"),
+        "roofline": {"bound": "tensor", "kernel": "attn::attn_fwd_kernel<128, false>",
                      "achieved": pf_tflops_1, "peak": meas_tf, "unit": "TFLOP/s", "frac": pf_tflops_1 / meas_tf,
                      "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
                      "traffic": ncu_traffic(P.name), "traffic_source": "ncu dram__bytes_read.sum + "
@@ -411,7 +413,7 @@ def run_ours(args, world, rank, local, dist):
         "e2e": {"value": world * pf_flops / (e2e["ms"] * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
         "gates": gates,
-        "gpu_launches": 3 * K,
+        "gpu_launches": 3 * K,  # per step: the prefill kernel, the decode split kernel, the combine kernel
         "kernels": {"prefill": lib.kernel_name(0), "decode": [lib.kernel_name(1), lib.kernel_name(2)]},
         "clocks": clocks,
         "cpu_baseline": cpu,
@@ -453,9 +455,61 @@ def time_prefill(lib, w, dev, stream, peaks, reps=20, warm=5):
     tf = w.flops / (med * 1e-3) / 1e12
     pk = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
     return {"ms": med, "tflops": tf, "frac_of_measured": tf / pk, "frac_of_nominal": tf / NOMINAL_BF16_TFLOPS,
-            "roofline": {"bound": "tensor", "kernel": f"attn::attn_fwd_kernel<{w.d}>", "achieved": tf, "peak": pk,
+            "roofline": {"bound": "tensor", "kernel": f"attn::attn_fwd_kernel<{w.d}, false>", "achieved": tf, "peak": pk,
                          "unit": "TFLOP/s", "frac": tf / pk, "traffic": ncu_traffic(w.name),
                          "algorithmic_bytes": prefill_bytes(w)}}
+
+
+FP8_SIGNS_SEED = 4242
+
+
+def fp8_signs(d: int, device):
+    """The rotation's sign vector: +-1 from a seeded generator (an input of the method)."""
+    import torch
+
+    u = np.random.default_rng(FP8_SIGNS_SEED).random(d)
+    return torch.from_numpy(np.where(u < 0.5, -1.0, 1.0).astype(np.float32)).to(device)
+
+
+def time_prefill_fp8(lib, w, dev, stream, peaks, reps=20, warm=5):
+    """attn_fwd_fp8 on the workload's inputs quantized once (rotation + e4m3, not timed), one launch
+    at a time after an L2 flush; TFLOP/s against the fp8 dense peak (2x the measured bf16 peak, the
+    nominal fp8 / bf16 ratio)."""
+    import torch
+
+    q = synth.normal_bf16_torch(w.seed, synth.STREAM_Q, (w.B, w.Nq, w.Hq, w.d), dev)
+    k = synth.normal_bf16_torch(w.seed, synth.STREAM_K, (w.B, w.Nkv, w.Hkv, w.d), dev)
+    v = synth.normal_bf16_torch(w.seed, synth.STREAM_V, (w.B, w.Nkv, w.Hkv, w.d), dev)
+    sg = fp8_signs(w.d, dev)
+    q8, aq = lib.attn_fp8_quantize(q, sg)
+    k8, ak = lib.attn_fp8_quantize(k, sg)
+    vt8, av = lib.attn_fp8_quantize(v, None, transpose=True)
+    del q, k, v
+    o = torch.empty((w.B, w.Nq, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def call():
+        lib.attn_fwd_fp8(q8, k8, vt8, aq, ak, av, scale=w.scale, causal=w.causal, out=o, lse=lse)
+    for _ in range(warm):
+        call()
+    ms = []
+    for _ in range(reps):
+        flush.fill_(1)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        call()
+        b.record(stream)
+        b.synchronize()
+        ms.append(a.elapsed_time(b))
+    med = float(np.median(ms))
+    tf = w.flops / (med * 1e-3) / 1e12
+    pk = 2.0 * peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
+    return {"ms": med, "tflops": tf, "dtype": "e4m3 operands, fp32 accumulate",
+            "roofline": {"bound": "tensor", "kernel": "attn::attn_fwd_kernel<128, true>", "achieved": tf, "peak": pk,
+                         "unit": "TFLOP/s", "frac": tf / pk, "peak_source": "2 x bf16 peak (nominal fp8/bf16 ratio)",
+                         "traffic": ncu_traffic("fp8 " + w.name)}}
 
 
 def e2e_prefill(lib, P, q, k, v, stream, n):
@@ -649,7 +703,23 @@ def run_only(args):
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream()
     peaks, src = _peaks()
-    if args.only == "prefill":
+    if args.only == "prefill_fp8":
+        w = synth.LONG_8K
+        q = synth.normal_bf16_torch(w.seed, synth.STREAM_Q, (w.B, w.Nq, w.Hq, w.d), dev)
+        k = synth.normal_bf16_torch(w.seed, synth.STREAM_K, (w.B, w.Nkv, w.Hkv, w.d), dev)
+        v = synth.normal_bf16_torch(w.seed, synth.STREAM_V, (w.B, w.Nkv, w.Hkv, w.d), dev)
+        sg = fp8_signs(w.d, dev)
+        q8, aq = lib.attn_fp8_quantize(q, sg)
+        k8, ak = lib.attn_fp8_quantize(k, sg)
+        vt8, av = lib.attn_fp8_quantize(v, None, transpose=True)
+        del q, k, v
+        o = torch.empty((w.B, w.Nq, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+
+        def call():
+            lib.attn_fwd_fp8(q8, k8, vt8, aq, ak, av, scale=w.scale, causal=w.causal, out=o, lse=lse)
+        work, unit, name = w.flops / 1e12, "TFLOP/s", "fp8 " + w.name
+    elif args.only == "prefill":
         table = {w.name: w for w in synth.PREFILL_WORKLOADS}
         w = table[args.workload] if args.workload else synth.LONG_8K
         q = synth.normal_bf16_torch(w.seed, synth.STREAM_Q, (w.B, w.Nq, w.Hq, w.d), dev)
@@ -708,7 +778,7 @@ def main():
     ap.add_argument("--no-gates", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e-decode", action="store_true")
-    ap.add_argument("--only", choices=("prefill", "decode"), default=None,
+    ap.add_argument("--only", choices=("prefill", "prefill_fp8", "decode"), default=None,
                     help="time one kernel on one workload (profiling and per-workload numbers)")
     ap.add_argument("--workload", default=None, help="prefill workload name for --only prefill")
     ap.add_argument("--decode-cap", type=int, default=0, help="cap decode lengths/cache for --only decode")

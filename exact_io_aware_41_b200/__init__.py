@@ -39,6 +39,8 @@ SIGNATURES = {
     "attn_kernel_name": (ctypes.c_char_p, [_I]),
     "attn_selftest_bounded_wait": (_I, [ctypes.c_uint, _P]),
     "attn_selftest_exp2_poly": (_I, [_P, _P, _I, _P]),
+    "attn_fp8_quantize": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "attn_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
 }
 
 
@@ -232,3 +234,53 @@ def attn_selftest_exp2_poly(x, out=None, stream=None):
     _check("attn_selftest_exp2_poly",
            lib_handle().attn_selftest_exp2_poly(x.data_ptr(), out.data_ptr(), x.numel(), _stream(stream)))
     return out
+
+
+def attn_fp8_quantize(x, signs=None, transpose: bool = False, out=None, amax=None, stream=None):
+    """e4m3 codes of x [B, N, H, d] (bf16, d = 128) with per-(batch, head) maxima.
+
+    signs: fp32 [d] of +-1 (CUDA) to rotate by diag(signs) H / sqrt(d) first (Q and K), or None (V).
+    transpose: write codes as [B, H, d, N] (the layout attn_fwd_fp8 takes V in; N % 16 == 0).
+    Returns (codes uint8, amax fp32 [B, H]).
+    """
+    import torch
+
+    _bf16_cuda("x", x, 4)
+    B, N, H, d = x.shape
+    if signs is not None and (signs.dtype != torch.float32 or not signs.is_cuda or signs.shape != (d,)):
+        raise ValueError("signs must be a fp32 CUDA tensor of shape [d]")
+    if out is None:
+        out = torch.empty((B, H, d, N) if transpose else (B, N, H, d), dtype=torch.uint8, device=x.device)
+    if amax is None:
+        amax = torch.empty((B, H), dtype=torch.float32, device=x.device)
+    code = lib_handle().attn_fp8_quantize(x.data_ptr(), None if signs is None else signs.data_ptr(), out.data_ptr(),
+                                          amax.data_ptr(), B, N, H, d, int(bool(transpose)), _stream(stream))
+    _check("attn_fp8_quantize", code)
+    return out, amax
+
+
+def attn_fwd_fp8(q8, k8, vt8, amax_q, amax_k, amax_v, scale: float | None = None, causal: bool = False, out=None,
+                 lse=None, stream=None):
+    """8-bit prefill forward. q8 [B, Nq, Hq, d], k8 [B, Nkv, Hkv, d] (rotated codes), vt8 [B, Hkv, d, Nkv]
+    (transposed V codes), amax_* fp32 [B, H] from attn_fp8_quantize. Returns (O bf16 [B, Nq, Hq, d],
+    LSE fp32 [B, Hq, Nq])."""
+    import torch
+
+    for n, t in (("q8", q8), ("k8", k8), ("vt8", vt8)):
+        if t.dtype != torch.uint8 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{n} must be a contiguous 4-d uint8 CUDA tensor")
+    B, Nq, Hq, d = q8.shape
+    _, Nkv, Hkv, _ = k8.shape
+    if vt8.shape != (B, Hkv, d, Nkv):
+        raise ValueError("vt8 must be [B, Hkv, d, Nkv]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, Nq, Hq, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q8.device)
+    code = lib_handle().attn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), vt8.data_ptr(), amax_q.data_ptr(), amax_k.data_ptr(),
+                                     amax_v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, Nq, Nkv, d,
+                                     float(scale), int(bool(causal)), _stream(stream))
+    _check("attn_fwd_fp8", code)
+    return out, lse

@@ -50,20 +50,22 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-static bool encode_tile_map_uncached(CUtensorMap* map, const void* base, int d, int heads, int rows, int outer,
-                                     int box_cols, int box_rows, unsigned swizzle_bytes) {
+// A 4-d tiled TMA map: dims[0] innermost (contiguous), dims[i] elements of elem_bytes each, dense
+// strides; box[] elements per dimension; swizzle 128, 64 or 0 bytes.
+static bool encode_map_uncached(CUtensorMap* map, const void* base, int elem_bytes, const long long* dims,
+                                const int* box, unsigned swizzle_bytes) {
   auto fn = get_encode_fn();
   if (fn == nullptr) return false;
-  const cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(heads), cuuint64_t(rows), cuuint64_t(outer)};
-  const cuuint64_t strides[3] = {cuuint64_t(d) * 2, cuuint64_t(heads) * d * 2, cuuint64_t(rows) * heads * d * 2};
-  const cuuint32_t box[4] = {cuuint32_t(box_cols), 1u, cuuint32_t(box_rows), 1u};
+  const cuuint64_t gd[4] = {cuuint64_t(dims[0]), cuuint64_t(dims[1]), cuuint64_t(dims[2]), cuuint64_t(dims[3])};
+  const cuuint64_t gs[3] = {gd[0] * elem_bytes, gd[0] * gd[1] * elem_bytes, gd[0] * gd[1] * gd[2] * elem_bytes};
+  const cuuint32_t bx[4] = {cuuint32_t(box[0]), cuuint32_t(box[1]), cuuint32_t(box[2]), cuuint32_t(box[3])};
   const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
   const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                 : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
                                                       : CU_TENSOR_MAP_SWIZZLE_NONE;
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
-                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUresult r = fn(map, dt, 4, const_cast<void*>(base), gd, gs, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -72,11 +74,15 @@ namespace {
 // of the key, so a hit returns exactly the map the encoder would produce.
 struct MapKey {
   const void* base;
-  int d, heads, rows, outer, box_cols, box_rows;
+  int elem_bytes;
+  long long dims[4];
+  int box[4];
   unsigned swizzle;
   bool operator==(const MapKey& o) const {
-    return base == o.base && d == o.d && heads == o.heads && rows == o.rows && outer == o.outer &&
-           box_cols == o.box_cols && box_rows == o.box_rows && swizzle == o.swizzle;
+    if (base != o.base || elem_bytes != o.elem_bytes || swizzle != o.swizzle) return false;
+    for (int i = 0; i < 4; ++i)
+      if (dims[i] != o.dims[i] || box[i] != o.box[i]) return false;
+    return true;
   }
 };
 constexpr int kMapCacheSize = 64;
@@ -93,9 +99,9 @@ MapCache& map_cache() {
 }
 }  // namespace
 
-bool encode_tile_map(CUtensorMap* map, const void* base, int d, int heads, int rows, int outer, int box_cols,
-                     int box_rows, unsigned swizzle_bytes) {
-  const MapKey k{base, d, heads, rows, outer, box_cols, box_rows, swizzle_bytes};
+bool encode_map(CUtensorMap* map, const void* base, int elem_bytes, const long long* dims, const int* box,
+                unsigned swizzle_bytes) {
+  MapKey k{base, elem_bytes, {dims[0], dims[1], dims[2], dims[3]}, {box[0], box[1], box[2], box[3]}, swizzle_bytes};
   MapCache& c = map_cache();
   std::lock_guard<std::mutex> lock(c.mu);
   for (int i = 0; i < kMapCacheSize; ++i) {
@@ -104,13 +110,20 @@ bool encode_tile_map(CUtensorMap* map, const void* base, int d, int heads, int r
       return true;
     }
   }
-  if (!encode_tile_map_uncached(map, base, d, heads, rows, outer, box_cols, box_rows, swizzle_bytes)) return false;
+  if (!encode_map_uncached(map, base, elem_bytes, dims, box, swizzle_bytes)) return false;
   const int slot = c.next;
   c.next = (c.next + 1) % kMapCacheSize;
   c.key[slot] = k;
   c.map[slot] = *map;
   c.used[slot] = true;
   return true;
+}
+
+bool encode_tile_map(CUtensorMap* map, const void* base, int d, int heads, int rows, int outer, int box_cols,
+                     int box_rows, unsigned swizzle_bytes) {
+  const long long dims[4] = {d, heads, rows, outer};
+  const int box[4] = {box_cols, 1, box_rows, 1};
+  return encode_map(map, base, 2, dims, box, swizzle_bytes);
 }
 
 namespace {
@@ -175,6 +188,34 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   if (!(scale > 0.f) || !isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
   if (d != 32 && d != 64 && d != 128 && d != 256) return ATTN_ERR_UNSUPPORTED;
   return fwd_dispatch(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, stream);
+}
+
+attn_status_t attn_fp8_quantize(const void* x, const float* signs, void* codes, float* amax, int B, int N, int H,
+                                int d, int transpose, cudaStream_t stream) {
+  if (!x || !codes || !amax) return ATTN_ERR_INVALID_ARG;
+  if (!is_aligned16(x) || !is_aligned16(codes) || (reinterpret_cast<uintptr_t>(amax) & 3u) ||
+      (reinterpret_cast<uintptr_t>(signs) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H < 1 || (transpose != 0 && transpose != 1)) return ATTN_ERR_INVALID_ARG;
+  if (transpose && (N % 16) != 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * H > 65535) return ATTN_ERR_UNSUPPORTED;  // grid y
+  return fp8_quantize_dispatch(x, signs, codes, amax, B, N, H, transpose, stream);
+}
+
+attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* amax_q, const float* amax_k,
+                           const float* amax_v, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                           float scale, int causal, cudaStream_t stream) {
+  if (!q8 || !k8 || !vt8 || !amax_q || !amax_k || !amax_v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!is_aligned16(q8) || !is_aligned16(k8) || !is_aligned16(vt8) || !is_aligned16(o) || !is_aligned16(lse) ||
+      ((reinterpret_cast<uintptr_t>(amax_q) | reinterpret_cast<uintptr_t>(amax_k) |
+        reinterpret_cast<uintptr_t>(amax_v)) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
+  if (Nkv % 16 != 0) return ATTN_ERR_INVALID_ARG;  // rows of the transposed V start on 16-byte boundaries
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  return fwd_fp8_dispatch(q8, k8, vt8, amax_q, amax_k, amax_v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, stream);
 }
 
 int attn_decode_default_chunk(int B, int Hkv, int Nkv_cap) {
@@ -253,7 +294,7 @@ const char* attn_status_string(attn_status_t s) {
 
 const char* attn_kernel_name(int which) {
   switch (which) {
-    case 0: return "attn::attn_fwd_kernel<D>";
+    case 0: return "attn::attn_fwd_kernel<D, F8>";
     case 1: return "attn::decode_split_tc_kernel<D,G> (d <= 128), attn::decode_split_kernel<D,G> (d = 256)";
     case 2: return "attn::decode_combine_kernel<D>";
   }

@@ -65,8 +65,12 @@ constexpr float kRescaleTau = 8.0f;
 #define ATTN_EMU_COLS_D256 0
 #endif
 
-template <int D>
+// F8: Q and K are e4m3 codes (rotated), V is given transposed (e4m3 [d, keys] per head), and the
+// products run as kind::f8f6f4 MMAs with 32-element k-steps; P is packed four e4m3 per TMEM column.
+template <int D, bool F8 = false>
 struct FwdCfg {
+  static_assert(!F8 || D == 128, "the 8-bit path is built for d = 128");
+  static constexpr int EB = F8 ? 1 : 2;                 // bytes per element of Q, K, V
   static constexpr int BM = 128;                        // query rows per tile (TMEM lanes)
   static constexpr int NQT = (D <= 128) ? 2 : 1;        // query tiles per CTA
   static constexpr int BN = (D <= 128) ? 128 : 64;      // keys per K/V tile
@@ -74,15 +78,17 @@ struct FwdCfg {
   // S = Q K^T is computed while the softmax still works on the current one (the two O accumulators
   // leave room for the buffers). d = 128 has no room for them and writes P over S.
   static constexpr bool SEP_P = (NQT == 2) && (D < 128);
-  static constexpr int CHUNK = (D >= 64) ? 64 : 32;     // elements per swizzled smem row
+  static constexpr int CHUNK = (D * EB >= 128) ? 128 / EB : D;  // elements per swizzled smem row
   static constexpr int NCHUNK = D / CHUNK;              // swizzle chunks along d
-  static constexpr int ROWB = CHUNK * 2;                // bytes per swizzled row (128 or 64)
-  static constexpr uint32_t LAYOUT = (D >= 64) ? kLayoutSW128 : kLayoutSW64;
-  static constexpr int KPC = CHUNK / 16;                // 16-wide MMA k-steps per chunk
+  static constexpr int ROWB = CHUNK * EB;               // bytes per swizzled row (128 or 64)
+  static constexpr uint32_t LAYOUT = (ROWB == 128) ? kLayoutSW128 : kLayoutSW64;
+  static constexpr int KSTEP = 32 / EB;                 // elements per MMA k-step (32 bytes)
+  static constexpr int KPC = CHUNK / KSTEP;             // MMA k-steps per chunk
   static constexpr int Q_CHUNK_BYTES = BM * ROWB;
   static constexpr int KV_CHUNK_BYTES = BN * ROWB;
-  static constexpr int Q_TILE_BYTES = BM * D * 2;
-  static constexpr int KV_TILE_BYTES = BN * D * 2;
+  static constexpr int Q_TILE_BYTES = BM * D * EB;
+  static constexpr int KV_TILE_BYTES = BN * D * EB;
+  static_assert(!F8 || BN * EB == 128, "a transposed V tile row (BN keys) is one 128-byte swizzled row");
   static constexpr int STAGES = (D == 256) ? 5 : (KV_TILE_BYTES >= 32768) ? 4 : 8;
   static constexpr int NSMWG = (NQT == 2) ? 2 : 1;      // softmax warpgroups
   static constexpr int THREADS = 128 * (1 + NSMWG);
@@ -92,11 +98,11 @@ struct FwdCfg {
   static constexpr bool SPLIT_REGS = (NQT == 2);
   static constexpr int CTRL_REGS = 104;
   static constexpr int SM_REGS = 192;
-  static constexpr int EMU_COLS = D == 32 ? ATTN_EMU_COLS_D32 : D == 64 ? ATTN_EMU_COLS_D64
+  static constexpr int EMU_COLS = F8 ? 0 : D == 32 ? ATTN_EMU_COLS_D32 : D == 64 ? ATTN_EMU_COLS_D64
                                   : D == 128 ? ATTN_EMU_COLS_D128 : ATTN_EMU_COLS_D256;
   static_assert(EMU_COLS % 8 == 0 && EMU_COLS >= 0 && EMU_COLS <= 128, "emulated column count");
-  static constexpr int HALF_PAIRS = BN / 4;             // bf16 pairs (TMEM columns) of P per half tile
-  static constexpr int PV_KH = BN / 32;                 // PV k-steps (16 keys) per half tile
+  static constexpr int PPC = 4 / EB;                    // P values per 32-bit TMEM column (2 bf16, 4 e4m3)
+  static constexpr int HALF_PAIRS = BN / 2 / PPC;       // TMEM columns of P per half tile
   // TMEM columns (fp32 each): two S slots, then one O accumulator per query tile.
   static constexpr int S_COL0 = 0;
   static constexpr int S_COL1 = BN;
@@ -179,11 +185,11 @@ __device__ __forceinline__ Unit unit_at(const FwdArgs& a, int lin) {
   return u;
 }
 
-template <int D>
-__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
+template <int D, bool F8>
+__global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdArgs args) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
@@ -255,23 +261,27 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   constexpr bool kSplitRegs = C::SPLIT_REGS;
 
   // ---- MMA issue helpers ------------------------------------------------------------------------
-  constexpr uint32_t idesc_qk = idesc_bf16_f32(128, C::BN, 0, 0);
-  constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+  // bf16: V is read MN-major (rows of d); 8-bit: V is given transposed and read K-major like K
+  constexpr uint32_t idesc_qk = F8 ? idesc_e4m3_f32(128, C::BN, 0, 0) : idesc_bf16_f32(128, C::BN, 0, 0);
+  constexpr uint32_t idesc_pv = F8 ? idesc_e4m3_f32(128, D, 0, 0) : idesc_bf16_f32(128, D, 0, 1);
   // Only the start-address field (bits 0-13, 16-byte units) differs between the descriptors of one
   // operand, so each base descriptor is built once and the k-step offsets are added to it.
   // Shared-memory addresses stay below 2^18, so the field never carries into its neighbour.
   const uint64_t dQ = smem_desc(smem_u32(sQ), 16, 8 * C::ROWB, C::LAYOUT);
   const uint64_t dK = smem_desc(smem_u32(sKV), 16, 8 * C::ROWB, C::LAYOUT);
-  const uint64_t dV = smem_desc(smem_u32(sKV), C::KV_CHUNK_BYTES, 8 * C::ROWB, C::LAYOUT);
+  const uint64_t dV = F8 ? smem_desc(smem_u32(sKV), 16, 8 * C::ROWB, C::LAYOUT)
+                        : smem_desc(smem_u32(sKV), C::KV_CHUNK_BYTES, 8 * C::ROWB, C::LAYOUT);
   // S[slot] = Q_qt K^T : A = Q tile (K-major), B = K tile (K-major), k-steps of 16 along d.
   auto issue_qk = [&](int qt, int s_col, int stage) {
     const uint64_t a0 = dQ + uint64_t((qt * C::Q_TILE_BYTES) >> 4);
     const uint64_t b0 = dK + uint64_t((stage * C::KV_TILE_BYTES) >> 4);
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
+    for (int kk = 0; kk < D / C::KSTEP; ++kk) {
       const uint32_t ao = (kk / C::KPC) * C::Q_CHUNK_BYTES + (kk % C::KPC) * 32;
       const uint32_t bo = (kk / C::KPC) * C::KV_CHUNK_BYTES + (kk % C::KPC) * 32;
-      if (C::Q_TMEM)
+      if (F8)
+        umma_ss_f8(tmem + s_col, a0 + (ao >> 4), b0 + (bo >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+      else if (C::Q_TMEM)
         umma_ts(tmem + s_col, tmem + C::Q_COL + kk * 8, b0 + (bo >> 4), idesc_qk, kk > 0 ? 1u : 0u);
       else
         umma_ss(tmem + s_col, a0 + (ao >> 4), b0 + (bo >> 4), idesc_qk, kk > 0 ? 1u : 0u);
@@ -292,9 +302,16 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   auto issue_pv = [&](int o_col, int p_col, int stage, bool accumulate) {
     const uint64_t b0 = dV + uint64_t((stage * C::KV_TILE_BYTES) >> 4);
 #pragma unroll
-    for (int kk = 0; kk < C::BN / 16; ++kk)
-      umma_ts(tmem + o_col, tmem + p_col + kk * 8, b0 + uint64_t((kk * 16 * C::ROWB) >> 4), idesc_pv,
-              (accumulate || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < C::BN / C::KSTEP; ++kk) {
+      // A = P: KSTEP keys = 8 TMEM columns in both forms; B: the next KSTEP rows of V (MN-major) or
+      // the next 32 bytes of each transposed-V row (K-major)
+      if (F8)
+        umma_ts_f8(tmem + o_col, tmem + p_col + kk * 8, b0 + uint64_t((kk * 32) >> 4), idesc_pv,
+                   (accumulate || kk > 0) ? 1u : 0u);
+      else
+        umma_ts(tmem + o_col, tmem + p_col + kk * 8, b0 + uint64_t((kk * 16 * C::ROWB) >> 4), idesc_pv,
+                (accumulate || kk > 0) ? 1u : 0u);
+    }
   };
   // K/V ring positions run on across units; inside a unit K_j is at base + 2j, V_j at base + 2j + 1.
   auto kv_slot = [](int pos) { return pos % C::STAGES; };
@@ -360,10 +377,15 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             }
             mbar_arrive_expect_tx(&kv_full[s], C::KV_TILE_BYTES);
             const CUtensorMap* m = kv ? &tmV : &tmK;
+            if (F8 && kv) {
+              // transposed V [B, Hkv, d, Nkv]: keys j*BN .. j*BN+BN-1 of all d rows, one box
+              tma_load_4d(sKV + s * C::KV_TILE_BYTES, m, &kv_full[s], j * C::BN, 0, g, un.b);
+            } else {
 #pragma unroll
-            for (int c = 0; c < C::NCHUNK; ++c)
-              tma_load_4d(sKV + s * C::KV_TILE_BYTES + c * C::KV_CHUNK_BYTES, m, &kv_full[s], c * C::CHUNK, g,
-                          j * C::BN, un.b);
+              for (int c = 0; c < C::NCHUNK; ++c)
+                tma_load_4d(sKV + s * C::KV_TILE_BYTES + c * C::KV_CHUNK_BYTES, m, &kv_full[s], c * C::CHUNK, g,
+                            j * C::BN, un.b);
+            }
           }
         }
       }
@@ -555,7 +577,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     const int qt = (C::NQT == 2) ? wg : 0;
     const uint32_t lane_addr = tmem + (uint32_t(wq * 32) << 16);
     const uint32_t o_col = qt ? C::O_COL1 : C::O_COL0;
-    const float c = args.scale_log2;
+    float c = args.scale_log2;  // log2-domain factor on the raw scores (8-bit: times both dequantizations)
+    float sc_nat = args.scale;  // the same in natural-log units, for the LSE
+    float o_mul = 1.0f;         // epilogue factor on O (8-bit: V's dequantization)
     // every lane waits; the warp continues only if all of them saw the phase (tcgen05.ld/st below are
     // warp-collective, so a partial give-up must not split the warp)
     auto wait_warp = [&](uint64_t* bar, uint32_t ph) -> bool {
@@ -571,6 +595,15 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       const int lin = next_unit(k, true);
       if (lin < 0) break;
       const Unit un = unit_at<D>(args, lin);
+      if (F8) {
+        // codes decode as value = code * amax / 448 per (batch, head)
+        const int g = un.h / args.group;
+        const float dq = args.amax_q[un.b * args.Hq + un.h] / 448.0f;
+        const float dk = args.amax_k[un.b * args.Hkv + g] / 448.0f;
+        c = args.scale_log2 * dq * dk;
+        sc_nat = args.scale * dq * dk;
+        o_mul = args.amax_v[un.b * args.Hkv + g] / 448.0f;
+      }
       const int q_first = un.q0 + qt * C::BM;
       const int q_row = q_first + row;
       // last key visible to this row (any key index <= lim is visible); rows past Nq are padding
@@ -703,20 +736,37 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t p[C::HALF_PAIRS];
+          if constexpr (F8) {
+            // four keys per TMEM column, e4m3 (P <= 2^TAU stays far below the e4m3 limit of 448)
 #pragma unroll
-          for (int i2 = 0; i2 < C::HALF_PAIRS; ++i2) {
-            const int i = half * C::HALF_PAIRS + i2;
-            const float2 x =
-                ffma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nmc2);
-            float2 e;
-            if (i >= EMU_FROM && emu) {
-              e = exp2_poly2(x);
-            } else {
-              e.x = ex2(x.x);
-              e.y = ex2(x.y);
+            for (int i2 = 0; i2 < C::HALF_PAIRS; ++i2) {
+              const int k0 = 4 * (half * C::HALF_PAIRS + i2);
+              const float2 x0 =
+                  ffma2(make_float2(__uint_as_float(r[k0]), __uint_as_float(r[k0 + 1])), c2, nmc2);
+              const float2 x1 =
+                  ffma2(make_float2(__uint_as_float(r[k0 + 2]), __uint_as_float(r[k0 + 3])), c2, nmc2);
+              const float2 e0 = make_float2(ex2(x0.x), ex2(x0.y));
+              const float2 e1 = make_float2(ex2(x1.x), ex2(x1.y));
+              acc4[(2 * i2) & 3] = fadd2(acc4[(2 * i2) & 3], e0);
+              acc4[(2 * i2 + 1) & 3] = fadd2(acc4[(2 * i2 + 1) & 3], e1);
+              p[i2] = pack_e4m3x4(e0.x, e0.y, e1.x, e1.y);
             }
-            acc4[i & 3] = fadd2(acc4[i & 3], e);
-            p[i2] = pack_bf16x2(e.x, e.y);
+          } else {
+#pragma unroll
+            for (int i2 = 0; i2 < C::HALF_PAIRS; ++i2) {
+              const int i = half * C::HALF_PAIRS + i2;
+              const float2 x =
+                  ffma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), c2, nmc2);
+              float2 e;
+              if (i >= EMU_FROM && emu) {
+                e = exp2_poly2(x);
+              } else {
+                e.x = ex2(x.x);
+                e.y = ex2(x.y);
+              }
+              acc4[i & 3] = fadd2(acc4[i & 3], e);
+              p[i2] = pack_bf16x2(e.x, e.y);
+            }
           }
           if (C::HALF_PAIRS == 32)
             tmem_st32(p_addr + half * C::HALF_PAIRS, p);
@@ -754,7 +804,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         }
         ++uc;
         tc_fence_after();
-        const float inv = (l > 0.f) ? 1.0f / l : 0.f;
+        const float inv = (l > 0.f) ? o_mul / l : 0.f;
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
@@ -780,7 +830,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       }
       if (valid)
         args.lse[(size_t(un.b) * args.Hq + un.h) * args.Nq + q_row] =
-            (l > 0.f) ? fmaf(m_ref, args.scale, logf(l)) : -INFINITY;
+            (l > 0.f) ? fmaf(m_ref, sc_nat, logf(l)) : -INFINITY;
     }
   }
 
@@ -803,18 +853,28 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 // ---------------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------------
-template <int D>
+// F8: q and k are e4m3 codes [B, N, H, d], v is the transposed code tensor [B, Hkv, d, Nkv] and
+// amax_* the per-(batch, head) dequantization maxima; otherwise bf16 tensors and null amax.
+template <int D, bool F8>
 static attn_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                                int Hkv, int Nq, int Nkv, float scale, int causal, cudaStream_t stream) {
-  using C = FwdCfg<D>;
+                                int Hkv, int Nq, int Nkv, float scale, int causal, const float* amax_q,
+                                const float* amax_k, const float* amax_v, cudaStream_t stream) {
+  using C = FwdCfg<D, F8>;
   CUtensorMap tmQ, tmK, tmV;
-  const uint32_t swz = (D >= 64) ? 128u : 64u;
-  if (!encode_tile_map(&tmQ, q, D, Hq, Nq, B, C::CHUNK, C::BM, swz) ||
-      !encode_tile_map(&tmK, k, D, Hkv, Nkv, B, C::CHUNK, C::BN, swz) ||
-      !encode_tile_map(&tmV, v, D, Hkv, Nkv, B, C::CHUNK, C::BN, swz))
+  const uint32_t swz = C::ROWB == 128 ? 128u : 64u;
+  if (F8) {
+    const long long dq[4] = {D, Hq, Nq, B}, dk[4] = {D, Hkv, Nkv, B}, dvt[4] = {Nkv, D, Hkv, B};
+    const int bq[4] = {C::CHUNK, 1, C::BM, 1}, bk[4] = {C::CHUNK, 1, C::BN, 1}, bv[4] = {C::BN, D, 1, 1};
+    if (!encode_map(&tmQ, q, 1, dq, bq, swz) || !encode_map(&tmK, k, 1, dk, bk, swz) ||
+        !encode_map(&tmV, v, 1, dvt, bv, swz))
+      return ATTN_ERR_CUDA;
+  } else if (!encode_tile_map(&tmQ, q, D, Hq, Nq, B, C::CHUNK, C::BM, swz) ||
+             !encode_tile_map(&tmK, k, D, Hkv, Nkv, B, C::CHUNK, C::BN, swz) ||
+             !encode_tile_map(&tmV, v, D, Hkv, Nkv, B, C::CHUNK, C::BN, swz)) {
     return ATTN_ERR_CUDA;
+  }
 
-  if (ensure_dyn_smem(reinterpret_cast<const void*>(attn_fwd_kernel<D>), C::SMEM_BYTES) != cudaSuccess)
+  if (ensure_dyn_smem(reinterpret_cast<const void*>(attn_fwd_kernel<D, F8>), C::SMEM_BYTES) != cudaSuccess)
     return ATTN_ERR_CUDA;
   // setmaxnreg.inc waits until the registers it asks for are free in the CTA's launch allocation,
   // so a split whose total exceeds that allocation would never proceed: refuse to launch it.
@@ -823,7 +883,7 @@ static attn_status_t launch_fwd(const void* q, const void* k, const void* v, voi
     int st = regs_ok.load(std::memory_order_relaxed);
     if (st == 0) {
       cudaFuncAttributes fa;
-      if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D>) != cudaSuccess) return ATTN_ERR_CUDA;
+      if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, F8>) != cudaSuccess) return ATTN_ERR_CUDA;
       const long long pool = (long long)fa.numRegs * C::THREADS;
       const long long need = 128LL * C::CTRL_REGS + 128LL * C::NSMWG * C::SM_REGS;
       st = pool >= need ? 1 : 2;
@@ -845,13 +905,16 @@ static attn_status_t launch_fwd(const void* q, const void* k, const void* v, voi
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.timeout_ns = kWaitLimitNs;
+  a.amax_q = amax_q;
+  a.amax_k = amax_k;
+  a.amax_v = amax_v;
   // heads per L2 group: K/V of one kv head is read by every query head of its group and block; keep
   // a group's K/V within ~48 MB of the 126 MB L2. Causal launches whose K/V fits in L2 comfortably
   // use one group: longest-first then runs over every unit, so no group's long units start near the
   // end of the launch.
   {
-    const double kv_bytes_per_head = 2.0 * Nkv * D * 2 / double(Hq / Hkv);
-    const double kv_bytes_total = 2.0 * Nkv * D * 2 * double(B) * Hkv;
+    const double kv_bytes_per_head = 2.0 * Nkv * D * C::EB / double(Hq / Hkv);
+    const double kv_bytes_total = 2.0 * Nkv * D * C::EB * double(B) * Hkv;
     long long gh = (causal && kv_bytes_total <= kL2OneGroupBytes) ? (long long)B * Hq
                                                                   : (long long)(48.0e6 / kv_bytes_per_head);
     if (gh < 1) gh = 1;
@@ -866,19 +929,27 @@ static attn_status_t launch_fwd(const void* q, const void* k, const void* v, voi
   const unsigned grid = unsigned(units < sms ? units : sms);
   static std::atomic<unsigned> launch_count{0};
   a.sched_slot = int(launch_count.fetch_add(1) % kSchedSlots);
-  attn_fwd_kernel<D><<<dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, a);
+  attn_fwd_kernel<D, F8><<<dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, a);
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
 }
 
 attn_status_t fwd_dispatch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                            int Hkv, int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream) {
   switch (d) {
-    case 32: return launch_fwd<32>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, stream);
-    case 64: return launch_fwd<64>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, stream);
-    case 128: return launch_fwd<128>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, stream);
-    case 256: return launch_fwd<256>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, stream);
+    case 32: return launch_fwd<32, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, nullptr, nullptr, nullptr, stream);
+    case 64: return launch_fwd<64, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, nullptr, nullptr, nullptr, stream);
+    case 128: return launch_fwd<128, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, nullptr, nullptr, nullptr, stream);
+    case 256: return launch_fwd<256, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, nullptr, nullptr, nullptr, stream);
     default: return ATTN_ERR_UNSUPPORTED;
   }
+}
+
+attn_status_t fwd_fp8_dispatch(const void* q8, const void* k8, const void* vt8, const float* amax_q,
+                               const float* amax_k, const float* amax_v, void* o, float* lse, int B, int Hq, int Hkv,
+                               int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream) {
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  return launch_fwd<128, true>(q8, k8, vt8, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, amax_q, amax_k, amax_v,
+                               stream);
 }
 
 }  // namespace attn

@@ -30,6 +30,9 @@ struct FwdArgs {
   float scale;       // natural-log scale on Q K^T
   float scale_log2;  // scale * log2(e)
   unsigned long long timeout_ns;
+  const float* amax_q;  // 8-bit path: per-(batch, head) maxima the codes were scaled by; else null
+  const float* amax_k;
+  const float* amax_v;
 };
 
 bool is_aligned16(const void* p);
@@ -47,6 +50,11 @@ int sm_count();
 bool encode_tile_map(CUtensorMap* map, const void* base, int d, int heads, int rows, int outer, int box_cols,
                      int box_rows, unsigned swizzle_bytes);
 
+// The general form: a 4-d tensor of elem_bytes-sized elements (1: 8-bit codes, 2: bf16) with dense
+// strides, dims[0] innermost, box[] elements per dimension; cached like encode_tile_map.
+bool encode_map(CUtensorMap* map, const void* base, int elem_bytes, const long long* dims, const int* box,
+                unsigned swizzle_bytes);
+
 // Opts `func` into `bytes` of dynamic shared memory on the current device. The attribute belongs to
 // the function on one device, so it is set once per (function, device) and again only when a
 // larger size is asked for; safe to call from several host threads.
@@ -61,6 +69,12 @@ inline bool combine_fits(long long n_splits) {
 
 attn_status_t fwd_dispatch(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                            int Hkv, int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream);
+attn_status_t fwd_fp8_dispatch(const void* q8, const void* k8, const void* vt8, const float* amax_q,
+                               const float* amax_k, const float* amax_v, void* o, float* lse, int B, int Hq, int Hkv,
+                               int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream);
+
+attn_status_t fp8_quantize_dispatch(const void* x, const float* signs, void* codes, float* amax, int B, int N, int H,
+                                    int transpose, cudaStream_t stream);
 
 int decode_default_chunk(int B, int Hkv, int Nkv_cap);
 size_t decode_workspace(int B, int Hq, int d, int Nkv_cap, int chunk);

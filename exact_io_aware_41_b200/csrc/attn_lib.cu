@@ -5,3 +5,4 @@
 #include "attn_fwd.cu"
 #include "attn_decode.cu"
 #include "attn_decode_static.cu"
+#include "attn_fp8.cu"

@@ -69,6 +69,41 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
                        int Hkv, int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream);
 
 /*
+ * 8-bit inputs for attn_fwd_fp8, with incoherent processing (FP8 with incoherent processing:
+ * "Flash Attention" overview, FA-3 paragraph; FlashAttention generation comparison record, FA-3
+ * "Workarounds"). For each row of x (bf16 [B, N, H, d], d = 128), in fp32 and in this order:
+ *   y = x * signs (elementwise; skipped, with the next two steps, when signs is NULL);
+ *   fast Walsh-Hadamard butterflies (a, b) -> (a + b, a - b) for h = 1, 2, 4, ..., 64 on the pairs
+ *   (j, j + h) inside blocks of 2h (the Sylvester Hadamard matrix); y *= fp32(1 / sqrt(d));
+ * then amax[b, h] = max |y| over the head's rows and codes = e4m3(y * fp32(448 / amax[b, h]))
+ * (round to nearest even, saturating at +-448; scale 1 when amax = 0). A rotation is orthogonal, so
+ * rotating Q and K with the same signs leaves Q K^T unchanged while spreading outlier channels.
+ *   x      bf16 [B, N, H, d], read only;  signs fp32 [d] of +1 / -1 (device) or NULL
+ *   codes  uint8 (e4m3), written: [B, N, H, d], or [B, H, d, N] when transpose = 1 (the layout
+ *          attn_fwd_fp8 takes V in; then N must be a multiple of 16)
+ *   amax   fp32 [B, H], written (first zeroed on the stream, then raised by the kernels)
+ *   B, N, H >= 1, B * H <= 65535; d = 128 (ATTN_ERR_UNSUPPORTED otherwise).
+ */
+attn_status_t attn_fp8_quantize(const void* x, const float* signs, void* codes, float* amax, int B, int N, int H,
+                                int d, int transpose, cudaStream_t stream);
+
+/*
+ * Prefill forward on 8-bit operands: O = softmax(scale * Q' K'^T) V' and LSE, where Q', K', V' are
+ * the values the codes stand for (code value * amax / 448 per batch and head). The products run on
+ * the tensor cores in e4m3 (kind::f8f6f4) with fp32 accumulation; P is rounded to e4m3 before the PV
+ * product; softmax state, row sums and LSE are fp32 as in attn_fwd.
+ *   q8     uint8 [B, Nq, Hq, d] codes of Q (rotated), k8 uint8 [B, Nkv, Hkv, d] codes of K (rotated
+ *          with the same signs), vt8 uint8 [B, Hkv, d, Nkv] codes of V, transposed
+ *   amax_q fp32 [B, Hq], amax_k, amax_v fp32 [B, Hkv] as attn_fp8_quantize wrote them
+ *   o      bf16 [B, Nq, Hq, d], lse fp32 [B, Hq, Nq], written
+ *   d = 128 (ATTN_ERR_UNSUPPORTED otherwise); Nkv a multiple of 16 (ATTN_ERR_INVALID_ARG otherwise);
+ *   everything else as attn_fwd.
+ */
+attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* amax_q, const float* amax_k,
+                           const float* amax_v, void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nkv, int d,
+                           float scale, int causal, cudaStream_t stream);
+
+/*
  * Bytes of device workspace attn_decode_splitkv needs: the per-split partial outputs
  * (fp32 [B, Hq, n_splits, d]) and partial LSEs (fp32 [B, Hq, n_splits]), n_splits =
  * ceil(Nkv_cap / chunk). chunk = 0 selects the same automatic chunk attn_decode_splitkv uses.
@@ -160,8 +195,8 @@ attn_status_t attn_get_last_error(void);
 const char* attn_status_string(attn_status_t status);
 
 /*
- * Name of the kernel(s) that `which` selects (0 = prefill forward, 1 = decode split, 2 = decode
- * combine), for recording which kernel a measurement ran (the evolution article's section 1.1
+ * Name of the kernel(s) that `which` selects (0 = prefill forward, bf16 or 8-bit, 1 = decode split,
+ * 2 = decode combine), for recording which kernel a measurement ran (the evolution article's section 1.1
  * asks that a benchmark name its kernel). Returns NULL for an unknown index.
  */
 const char* attn_kernel_name(int which);

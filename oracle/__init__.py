@@ -228,3 +228,89 @@ def merge_partials(parts):
     z = w.sum()
     o = sum(wi * p[0] for wi, p in zip(w, parts)) / z
     return o, mx + np.log(z)
+
+
+# ------------------------------------------------------------------------------------------------
+# 8-bit path: incoherent processing and e4m3 quantization, then attention on the decoded values.
+# FP8 with incoherent processing is named by the "Flash Attention" overview (FA-3 paragraph) and the
+# FlashAttention generation comparison record (FA-3 "Workarounds"); the pages give no recipe, so the
+# steps below are this library's reading: rotate Q and K by diag(s) H / sqrt(d) (H the Sylvester
+# Hadamard matrix, s a sign vector), scale each (batch, head) so its largest |value| maps to 448,
+# round to e4m3 (nearest even, saturating). Q K^T is unchanged by the rotation in exact arithmetic.
+# The codes are an encoding, so the oracle follows the same fp32 steps in the same order (the
+# butterfly stages of the fast Walsh-Hadamard transform, then the fp32 products); the attention on
+# the decoded values is the plain definition above, in fp64.
+# ------------------------------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each e4m3 code (uint8): sign bit 7, exponent bits 6-3 (bias 7), mantissa bits 2-0;
+    exponent 0 is subnormal (m/8 * 2^-6); 0x7F / 0xFF are NaN (no infinities)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * 2.0 ** (e - 7.0))
+    val = np.where((c & 0x7F) == 0x7F, np.nan, val)
+    return sign * val
+
+
+_E4M3_GRID = None
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Codes of fp32 values rounded to the nearest e4m3 value (ties to the even code), saturating
+    at +-448; x must be finite."""
+    global _E4M3_GRID
+    if _E4M3_GRID is None:
+        pos = np.arange(0, 0x7F, dtype=np.uint8)            # 0 .. 0x7E: +0 .. 448, increasing
+        _E4M3_GRID = (pos, e4m3_decode(pos))
+    pos, grid = _E4M3_GRID
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.searchsorted(grid, a, side="left")               # first grid value >= a
+    hi = np.minimum(hi, len(grid) - 1)
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - grid[lo], grid[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (pos[hi] % 2 == 0))
+    idx = np.where(a == grid[hi], hi, np.where(pick_hi, hi, lo))
+    code = pos[idx].astype(np.uint8)
+    return np.where(np.signbit(x), code | 0x80, code).astype(np.uint8)  # the sign survives rounding to 0
+
+
+def hadamard_rotate_f32(x, signs) -> np.ndarray:
+    """Rows of x (last axis d, a power of two) times diag(signs) H / sqrt(d), in fp32: sign flip,
+    butterflies (a, b) -> (a + b, a - b) for h = 1, 2, ..., d/2 on pairs (j, j + h) inside blocks of
+    2h, then one fp32 product with fp32(1/sqrt(d))."""
+    y = np.asarray(x, dtype=np.float32) * np.asarray(signs, dtype=np.float32)
+    d = y.shape[-1]
+    lead = y.shape[:-1]
+    h = 1
+    while h < d:
+        z = y.reshape(lead + (d // (2 * h), 2, h))
+        a, b = z[..., 0, :], z[..., 1, :]
+        y = np.stack((a + b, a - b), axis=-2).reshape(lead + (d,)).astype(np.float32)
+        h *= 2
+    return (y * np.float32(1.0 / np.sqrt(d))).astype(np.float32)
+
+
+def fp8_quantize(x, signs=None):
+    """Codes and per-head maxima of x [B, N, H, d] (values exactly representable in fp32, e.g. bf16).
+
+    Returns (codes uint8 [B, N, H, d], amax fp32 [B, H]); code = e4m3(fp32(y * fp32(448 / amax)))
+    with y the rotated rows (or x itself without signs) and amax = max |y| over the head (scale 1
+    when amax = 0)."""
+    y = np.asarray(x, dtype=np.float32)
+    if signs is not None:
+        y = hadamard_rotate_f32(y, signs)
+    amax = np.abs(y).max(axis=(1, 3)).astype(np.float32)                      # [B, H]
+    scale = np.where(amax > 0, np.float32(E4M3_MAX) / np.where(amax > 0, amax, 1), 1).astype(np.float32)
+    codes = e4m3_round((y * scale[:, None, :, None]).astype(np.float32))
+    return codes, amax
+
+
+def fp8_dequantize(codes, amax) -> np.ndarray:
+    """Values the codes stand for: code value * amax / 448 per (batch, head), fp64; [B, N, H, d]."""
+    return e4m3_decode(codes) * (np.asarray(amax, dtype=np.float64) / E4M3_MAX)[:, None, :, None]
