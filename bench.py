@@ -351,6 +351,8 @@ def run_ours(args, world, rank, local, dist):
             torch.cuda.empty_cache()
         gates["fp8 " + P.name] = time_prefill_fp8(lib, P, dev, stream, peaks)
         torch.cuda.empty_cache()
+        gates["backward " + synth.CAUSAL_2K.name] = time_backward(lib, synth.CAUSAL_2K, dev, stream, peaks)
+        torch.cuda.empty_cache()
 
     # ---- end to end through the public API with pinned host buffers
     e2e = e2e_prefill(lib, P, q, k, v, stream, max(3, min(K, 50)))
@@ -510,6 +512,42 @@ def time_prefill_fp8(lib, w, dev, stream, peaks, reps=20, warm=5):
             "roofline": {"bound": "tensor", "kernel": "attn::attn_fwd_kernel<128, true>", "achieved": tf, "peak": pk,
                          "unit": "TFLOP/s", "frac": tf / pk, "peak_source": "2 x bf16 peak (nominal fp8/bf16 ratio)",
                          "traffic": ncu_traffic("fp8 " + w.name)}}
+
+
+def time_backward(lib, w, dev, stream, peaks, reps=20, warm=5):
+    """attn_bwd (pre-pass, main kernel, dQ conversion) after an L2 flush, on the forward's O and LSE.
+    FLOPs = 2.5 x the forward's (five products of the forward's size against two)."""
+    import torch
+
+    q = synth.normal_bf16_torch(w.seed, synth.STREAM_Q, (w.B, w.Nq, w.Hq, w.d), dev)
+    k = synth.normal_bf16_torch(w.seed, synth.STREAM_K, (w.B, w.Nkv, w.Hkv, w.d), dev)
+    v = synth.normal_bf16_torch(w.seed, synth.STREAM_V, (w.B, w.Nkv, w.Hkv, w.d), dev)
+    do = synth.normal_bf16_torch(w.seed, 5, (w.B, w.Nq, w.Hq, w.d), dev)
+    o, lse = lib.attn_fwd(q, k, v, scale=w.scale, causal=w.causal)
+    ws = torch.empty(lib.attn_bwd_workspace_bytes(w.B, w.Hq, w.Nq, w.d), dtype=torch.uint8, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def call():
+        lib.attn_bwd(q, k, v, o, lse, do, scale=w.scale, causal=w.causal, workspace=ws, dq=dq, dk=dk, dv=dv)
+    for _ in range(warm):
+        call()
+    ms = []
+    for _ in range(reps):
+        flush.fill_(1)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        call()
+        b.record(stream)
+        b.synchronize()
+        ms.append(a.elapsed_time(b))
+    med = float(np.median(ms))
+    tf = 2.5 * w.flops / (med * 1e-3) / 1e12
+    pk = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
+    return {"ms": med, "tflops": tf, "flops": 2.5 * w.flops,
+            "roofline": {"bound": "tensor", "kernel": "attn::attn_bwd_kernel (+ pre and post passes)", "achieved": tf,
+                         "peak": pk, "unit": "TFLOP/s", "frac": tf / pk, "traffic": ncu_traffic("backward " + w.name)}}
 
 
 def e2e_prefill(lib, P, q, k, v, stream, n):
@@ -703,7 +741,20 @@ def run_only(args):
     dev = torch.device("cuda", 0)
     stream = torch.cuda.current_stream()
     peaks, src = _peaks()
-    if args.only == "prefill_fp8":
+    if args.only == "backward":
+        w = synth.CAUSAL_2K
+        q = synth.normal_bf16_torch(w.seed, synth.STREAM_Q, (w.B, w.Nq, w.Hq, w.d), dev)
+        k = synth.normal_bf16_torch(w.seed, synth.STREAM_K, (w.B, w.Nkv, w.Hkv, w.d), dev)
+        v = synth.normal_bf16_torch(w.seed, synth.STREAM_V, (w.B, w.Nkv, w.Hkv, w.d), dev)
+        do = synth.normal_bf16_torch(w.seed, 5, (w.B, w.Nq, w.Hq, w.d), dev)
+        o, lse = lib.attn_fwd(q, k, v, scale=w.scale, causal=w.causal)
+        ws = torch.empty(lib.attn_bwd_workspace_bytes(w.B, w.Hq, w.Nq, w.d), dtype=torch.uint8, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+        def call():
+            lib.attn_bwd(q, k, v, o, lse, do, scale=w.scale, causal=w.causal, workspace=ws, dq=dq, dk=dk, dv=dv)
+        work, unit, name = 2.5 * w.flops / 1e12, "TFLOP/s", "backward " + w.name
+    elif args.only == "prefill_fp8":
         w = synth.LONG_8K
         q = synth.normal_bf16_torch(w.seed, synth.STREAM_Q, (w.B, w.Nq, w.Hq, w.d), dev)
         k = synth.normal_bf16_torch(w.seed, synth.STREAM_K, (w.B, w.Nkv, w.Hkv, w.d), dev)
@@ -778,7 +829,7 @@ def main():
     ap.add_argument("--no-gates", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e-decode", action="store_true")
-    ap.add_argument("--only", choices=("prefill", "prefill_fp8", "decode"), default=None,
+    ap.add_argument("--only", choices=("prefill", "prefill_fp8", "backward", "decode"), default=None,
                     help="time one kernel on one workload (profiling and per-workload numbers)")
     ap.add_argument("--workload", default=None, help="prefill workload name for --only prefill")
     ap.add_argument("--decode-cap", type=int, default=0, help="cap decode lengths/cache for --only decode")

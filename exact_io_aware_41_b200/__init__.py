@@ -41,6 +41,8 @@ SIGNATURES = {
     "attn_selftest_exp2_poly": (_I, [_P, _P, _I, _P]),
     "attn_fp8_quantize": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "attn_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
+    "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P, ctypes.c_size_t, _P]),
 }
 
 
@@ -284,3 +286,35 @@ def attn_fwd_fp8(q8, k8, vt8, amax_q, amax_k, amax_v, scale: float | None = None
                                      float(scale), int(bool(causal)), _stream(stream))
     _check("attn_fwd_fp8", code)
     return out, lse
+
+
+def attn_bwd_workspace_bytes(B: int, Hq: int, Nq: int, d: int) -> int:
+    return int(lib_handle().attn_bwd_workspace_bytes(B, Hq, Nq, d))
+
+
+def attn_bwd(q, k, v, o, lse, dout, scale: float | None = None, causal: bool = False, workspace=None, dq=None,
+             dk=None, dv=None, stream=None):
+    """Backward pass. q, o, dout [B, Nq, Hq, d], k, v [B, Nkv, Hkv, d] (bf16), lse fp32 [B, Hq, Nq] from
+    attn_fwd. Returns (dQ, dK, dV) in the layouts of q, k, v."""
+    import torch
+
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _bf16_cuda(n, t, 4)
+    B, Nq, Hq, d = q.shape
+    _, Nkv, Hkv, _ = k.shape
+    if o.shape != q.shape or dout.shape != q.shape or v.shape != k.shape or lse.shape != (B, Hq, Nq):
+        raise ValueError("o, dout like q; v like k; lse [B, Hq, Nq]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = attn_bwd_workspace_bytes(B, Hq, Nq, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    code = lib_handle().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                 dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Nq, Nkv, d,
+                                 float(scale), int(bool(causal)), workspace.data_ptr(),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("attn_bwd", code)
+    return dq, dk, dv

@@ -218,6 +218,29 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, cons
   return fwd_fp8_dispatch(q8, k8, vt8, amax_q, amax_k, amax_v, o, lse, B, Hq, Hkv, Nq, Nkv, d, scale, causal, stream);
 }
 
+size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq, int d) {
+  if (B < 1 || Hq < 1 || Nq < 1 || d < 1) return 0;
+  return bwd_workspace(B, Hq, Nq, d);
+}
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                       void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nkv, int d, float scale,
+                       int causal, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, dout, dq, dk, dv};
+  for (const void* p : ptrs)
+    if (!is_aligned16(p)) return ATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(lse) & 3u) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hq > 65535) return ATTN_ERR_UNSUPPORTED;  // grid y of the row passes
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < bwd_workspace(B, Hq, Nq, d))
+    return ATTN_ERR_WORKSPACE;
+  return bwd_dispatch(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Nq, Nkv, scale, causal, workspace, stream);
+}
+
 int attn_decode_default_chunk(int B, int Hkv, int Nkv_cap) {
   if (B < 1 || Hkv < 1 || Nkv_cap < 1) return 0;
   return decode_default_chunk(B, Hkv, Nkv_cap);
@@ -297,6 +320,7 @@ const char* attn_kernel_name(int which) {
     case 0: return "attn::attn_fwd_kernel<D, F8>";
     case 1: return "attn::decode_split_tc_kernel<D,G> (d <= 128), attn::decode_split_kernel<D,G> (d = 256)";
     case 2: return "attn::decode_combine_kernel<D>";
+    case 3: return "attn::attn_bwd_pre_kernel, attn::attn_bwd_kernel, attn::attn_bwd_post_kernel";
   }
   return nullptr;
 }

@@ -1,0 +1,457 @@
+// Backward pass for sm_100a (d = 128): dQ, dK, dV of O = softmax(scale * Q K^T) V, recomputing S tile
+// by tile instead of storing it (the FlashAttention generation comparison record, "Workarounds":
+// recompute S in backward). Per (batch, query head), with P = exp(scale * S - LSE):
+//   dV = P^T dO,  dP = dO V^T,  D = rowsum(dO * O),  dS = P * (dP - D),  dQ = scale dS K,
+//   dK = scale dS^T Q  (dK, dV of a kv head summed over the query heads of its group).
+//
+// One CTA per (key block of 128 keys, batch, kv head), heaviest key blocks first for causal masks.
+// It loads its K and V tiles once and walks every query head of its group and every query tile
+// that sees some of its keys. Per step (all products on tcgen05, accumulators in TMEM):
+//   S^T = K Q^T      (M = keys, N = queries)           -> TMEM columns [0, 128)
+//   dP^T = V dO^T                                      -> TMEM columns [128, 256)
+//   softmax warps (thread = key row): P^T = exp2(S^T * scale * log2 e - LSE * log2 e), masked;
+//   dS^T = P^T * (dP^T - D); P^T (bf16) over S^T, dS^T (bf16) over dP^T and into shared memory
+//   dV += P^T dO     (A = P^T in TMEM, B = dO read MN-major)   -> columns [256, 384), whole unit
+//   dK += dS^T Q     (A = dS^T in TMEM, B = Q read MN-major)   -> columns [384, 512), whole unit
+//   dQ  = dS K       (A = dS from shared memory, M-major; B = K read MN-major) -> columns [0, 128)
+//   the same warps add dQ (thread = query row) into an fp32 accumulator with vector atomics.
+// MMAs issued by one thread execute in issue order, so dQ may overwrite P^T's columns after the dV
+// product that reads them. The unit ends with dK (times scale) and dV stored as bf16.
+//
+// A pre-pass writes D and LSE * log2 e per query row (padded to whole tiles; rows without keys or
+// past Nq get LSE' = +inf, so their P is 0) and zeroes the dQ accumulator; a post-pass rounds
+// scale * dQ to bf16.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "attn_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace attn {
+
+namespace bwd {
+constexpr int D = 128;
+constexpr int BM = 128;                       // query rows per step
+constexpr int BN = 128;                       // keys per CTA
+constexpr int CHUNK_BYTES = 128 * 128;        // 64-column chunk of a 128-row tile (128-byte rows)
+constexpr int TILE_BYTES = 2 * CHUNK_BYTES;   // 128 x 128 bf16
+constexpr int THREADS = 256;
+constexpr int TMEM_COLS = 512;
+constexpr int S_COL = 0, DP_COL = 128, DV_COL = 256, DK_COL = 384;
+// shared memory: K, V, Q, dO, dS tiles, LSE' and D rows, barriers
+constexpr int OFF_K = 0, OFF_V = TILE_BYTES, OFF_Q = 2 * TILE_BYTES, OFF_DO = 3 * TILE_BYTES, OFF_DS = 4 * TILE_BYTES;
+constexpr int OFF_LSE = 5 * TILE_BYTES, OFF_DD = OFF_LSE + BM * 4, OFF_BAR = OFF_DD + BM * 4;
+constexpr int NBARS = 8;  // kv_full, q_full, q_empty, s_full, p_full, dq_full, dq_free, dkv_full
+constexpr int SMEM_BYTES = 1024 + OFF_BAR + NBARS * 8 + 16;
+}  // namespace bwd
+
+struct BwdArgs {
+  void* dk;
+  void* dv;
+  float* dq_acc;          // fp32 [B, Nq, Hq, d]
+  const float* lse2;      // [B * Hq, Nq_pad]: LSE * log2 e (+inf: no keys or padding)
+  const float* dd;        // [B * Hq, Nq_pad]: D
+  int B, Hq, Hkv, Nq, Nkv, Nq_pad, group, n_kb;
+  int causal;
+  float scale_log2;
+  float scale;
+  unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+// First query tile whose rows see some key of block kb (causal: key j visible to row i iff
+// j <= i + Nkv - Nq).
+__device__ __forceinline__ int first_q_tile(const BwdArgs& a, int kb) {
+  if (!a.causal) return 0;
+  const int lo = kb * bwd::BN - (a.Nkv - a.Nq);  // smallest row that sees key kb * BN
+  return lo <= 0 ? 0 : lo / bwd::BM;
+}
+
+__global__ void __launch_bounds__(bwd::THREADS, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                    const BwdArgs args) {
+  using namespace bwd;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;
+  uint64_t* q_empty = bars + 2;
+  uint64_t* s_full = bars + 3;
+  uint64_t* p_full = bars + 4;
+  uint64_t* dq_full = bars + 5;
+  uint64_t* dq_free = bars + 6;
+  uint64_t* dkv_full = bars + 7;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  const float* s_lse = reinterpret_cast<const float*>(smem + OFF_LSE);
+  const float* s_dd = reinterpret_cast<const float*>(smem + OFF_DD);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint64_t T = args.timeout_ns;
+  // unit: key block kb (heaviest first), batch b, kv head g
+  const int per_kb = args.B * args.Hkv;
+  const int kb = blockIdx.x / per_kb;
+  const int b = (blockIdx.x % per_kb) / args.Hkv;
+  const int g = blockIdx.x % args.Hkv;
+  const int n_qt = (args.Nq + BM - 1) / BM;
+  const int qt0 = first_q_tile(args, kb);
+  const int steps_per_head = qt0 < n_qt ? n_qt - qt0 : 0;
+  const int n_steps = steps_per_head * args.group;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NBARS; ++i) mbar_init(&bars[i], (i == 4 || i == 6) ? 4 : 1);  // p_full, dq_free: 4 warps
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_holder, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  // descriptors: K-major tiles (rows of d) and MN-major reads of the same tiles
+  const uint64_t dK_k = smem_desc(smem_u32(smem + OFF_K), 16, 1024, kLayoutSW128);
+  const uint64_t dV_k = smem_desc(smem_u32(smem + OFF_V), 16, 1024, kLayoutSW128);
+  const uint64_t dQ_k = smem_desc(smem_u32(smem + OFF_Q), 16, 1024, kLayoutSW128);
+  const uint64_t dDO_k = smem_desc(smem_u32(smem + OFF_DO), 16, 1024, kLayoutSW128);
+  const uint64_t dQ_mn = smem_desc(smem_u32(smem + OFF_Q), CHUNK_BYTES, 1024, kLayoutSW128);
+  const uint64_t dDO_mn = smem_desc(smem_u32(smem + OFF_DO), CHUNK_BYTES, 1024, kLayoutSW128);
+  const uint64_t dK_mn = smem_desc(smem_u32(smem + OFF_K), CHUNK_BYTES, 1024, kLayoutSW128);
+  const uint64_t dDS_mn = smem_desc(smem_u32(smem + OFF_DS), CHUNK_BYTES, 1024, kLayoutSW128);
+  constexpr uint32_t idesc_kk = idesc_bf16_f32(128, 128, 0, 0);   // A, B K-major
+  constexpr uint32_t idesc_tmn = idesc_bf16_f32(128, 128, 0, 1);  // A from TMEM, B MN-major
+  constexpr uint32_t idesc_mnmn = idesc_bf16_f32(128, 128, 1, 1); // A, B MN-major
+
+  auto step_coords = [&](int t, int& h, int& qt) {
+    h = g * args.group + t / steps_per_head;
+    qt = qt0 + t % steps_per_head;
+  };
+
+  if (warp == 0) {
+    // ================================ TMA producer ================================
+    if (lane == 0 && n_steps > 0) {
+      prefetch_tensormap(&tmQ);
+      prefetch_tensormap(&tmK);
+      prefetch_tensormap(&tmV);
+      prefetch_tensormap(&tmDO);
+      mbar_arrive_expect_tx(kv_full, 2 * TILE_BYTES);
+      for (int c = 0; c < 2; ++c) {
+        tma_load_4d(smem + OFF_K + c * CHUNK_BYTES, &tmK, kv_full, c * 64, g, kb * BN, b);
+        tma_load_4d(smem + OFF_V + c * CHUNK_BYTES, &tmV, kv_full, c * 64, g, kb * BN, b);
+      }
+      int t = 0;
+      for (; t < n_steps; ++t) {
+        if (t > 0 && !mbar_wait(q_empty, uint32_t((t - 1) & 1), abort_flag, T)) break;
+        int h, qt;
+        step_coords(t, h, qt);
+        mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES + 2 * BM * 4);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_4d(smem + OFF_Q + c * CHUNK_BYTES, &tmQ, q_full, c * 64, h, qt * BM, b);
+          tma_load_4d(smem + OFF_DO + c * CHUNK_BYTES, &tmDO, q_full, c * 64, h, qt * BM, b);
+        }
+        const size_t row = size_t(b * args.Hq + h) * args.Nq_pad + size_t(qt) * BM;
+        bulk_load(smem + OFF_LSE, args.lse2 + row, BM * 4, q_full);
+        bulk_load(smem + OFF_DD, args.dd + row, BM * 4, q_full);
+      }
+      // copies in flight land before the CTA exits (bounded)
+      mbar_wait(kv_full, 0, nullptr, 100000000ull);
+      if (t > 0) mbar_wait(q_full, uint32_t((t - 1) & 1), nullptr, 100000000ull);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ================================ MMA issuer ================================
+    if (lane == 0 && n_steps > 0) {
+      bool ok = mbar_wait(kv_full, 0, abort_flag, T);
+      for (int t = 0; t < n_steps && ok; ++t) {
+        ok = mbar_wait(q_full, uint32_t(t & 1), abort_flag, T);
+        if (ok && t > 0) ok = mbar_wait(dq_free, uint32_t((t - 1) & 1), abort_flag, T);  // columns [0, 128) read
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * CHUNK_BYTES + (kk % 4) * 32) >> 4;
+          umma_ss(tmem + S_COL, dK_k + off, dQ_k + off, idesc_kk, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * CHUNK_BYTES + (kk % 4) * 32) >> 4;
+          umma_ss(tmem + DP_COL, dV_k + off, dDO_k + off, idesc_kk, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full);
+        ok = mbar_wait(p_full, uint32_t(t & 1), abort_flag, T);
+        if (!ok) break;
+        tc_fence_after();
+        // over the step's 128 queries (k-steps of 16): dV += P^T dO, dK += dS^T Q, dQ = dS K
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          umma_ts(tmem + DV_COL, tmem + S_COL + kk * 8, dDO_mn + uint64_t((kk * 16 * 128) >> 4), idesc_tmn,
+                  (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          umma_ts(tmem + DK_COL, tmem + DP_COL + kk * 8, dQ_mn + uint64_t((kk * 16 * 128) >> 4), idesc_tmn,
+                  (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_ss(tmem + S_COL, dDS_mn + uint64_t((kk * 16 * 128) >> 4), dK_mn + uint64_t((kk * 16 * 128) >> 4),
+                  idesc_mnmn, kk > 0 ? 1u : 0u);
+        umma_commit(dq_full);
+        umma_commit(q_empty);
+        if (t == n_steps - 1) umma_commit(dkv_full);
+      }
+      if (!ok) {
+        // a wait gave up: let the MMAs already issued finish before tensor memory is released
+        // (dkv_full has not been committed on this path, so its first phase is the drain)
+        umma_commit(dkv_full);
+        mbar_wait(dkv_full, 0, nullptr, 100000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ========================= softmax / dQ / dK dV epilogue warps =========================
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;  // TMEM lane: key row (softmax, dK dV) or query row (dQ)
+    const uint32_t lane_addr = tmem + (uint32_t(wq * 32) << 16);
+    const float c = args.scale_log2;
+    const int key = kb * BN + row;
+    const bool key_ok = key < args.Nkv;
+    const int diag = args.Nkv - args.Nq;
+    auto wait_warp = [&](uint64_t* bar, uint32_t ph) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, ph, abort_flag, T));
+    };
+    bool ok = true;
+    for (int t = 0; t < n_steps && ok; ++t) {
+      int h, qt;
+      step_coords(t, h, qt);
+      if (!wait_warp(s_full, uint32_t(t & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int q0 = qt * BM;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {  // 32 query columns at a time
+        uint32_t sv[32], dpv[32];
+        tmem_ld32(lane_addr + S_COL + cc * 32, sv);
+        tmem_ld32(lane_addr + DP_COL + cc * 32, dpv);
+        tmem_ld_wait();
+        tmem_reg_fence32(sv);
+        tmem_reg_fence32(dpv);
+        uint32_t pk[16], dk2[16];
+#pragma unroll
+        for (int i2 = 0; i2 < 16; ++i2) {
+          float p2[2], ds2[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int qi = cc * 32 + 2 * i2 + u;
+            const int qrow = q0 + qi;
+            const bool vis = key_ok && (!args.causal || key <= qrow + diag);
+            const float p = vis ? ex2(fmaf(__uint_as_float(sv[2 * i2 + u]), c, -s_lse[qi])) : 0.f;
+            p2[u] = p;
+            ds2[u] = p * (__uint_as_float(dpv[2 * i2 + u]) - s_dd[qi]);
+          }
+          pk[i2] = pack_bf16x2(p2[0], p2[1]);
+          dk2[i2] = pack_bf16x2(ds2[0], ds2[1]);
+        }
+        // P^T over S^T and dS^T over dP^T (columns already read), both bf16 pairs
+        tmem_st16(lane_addr + S_COL + cc * 16, pk);
+        tmem_st16(lane_addr + DP_COL + cc * 16, dk2);
+        // dS^T row into the shared tile [key][query] (128-byte swizzled, 64-query chunks): the A
+        // operand of dQ = dS K, read M-major
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int qcol = cc * 32 + u * 8;
+          const int chunk = qcol >> 6, unit = (qcol & 63) >> 3;
+          const uint32_t addr =
+              smem_u32(smem + OFF_DS) + chunk * CHUNK_BYTES + row * 128 + ((unit ^ (row & 7)) << 4);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dk2[4 * u]), "r"(dk2[4 * u + 1]),
+                       "r"(dk2[4 * u + 2]), "r"(dk2[4 * u + 3])
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();  // the dS tile is read by the MMA (async proxy)
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+      // dQ of this step (thread = query row q0 + row): add into the fp32 accumulator
+      if (!wait_warp(dq_full, uint32_t(t & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int qrow = q0 + row;
+      float* dst = args.dq_acc + ((size_t(b) * args.Nq + (qrow < args.Nq ? qrow : 0)) * args.Hq + h) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(lane_addr + S_COL + cc * 32, o);
+        tmem_ld_wait();
+        tmem_reg_fence32(o);
+        if (qrow < args.Nq) {
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4)
+            red_add_v4(dst + cc * 32 + 4 * v4, __uint_as_float(o[4 * v4]), __uint_as_float(o[4 * v4 + 1]),
+                       __uint_as_float(o[4 * v4 + 2]), __uint_as_float(o[4 * v4 + 3]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_free);
+    }
+    // dK (times scale) and dV of this key block, bf16
+    if (key_ok) {
+      __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(args.dk) + ((size_t(b) * args.Nkv + key) * args.Hkv + g) * D;
+      __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(args.dv) + ((size_t(b) * args.Nkv + key) * args.Hkv + g) * D;
+      if (n_steps == 0) {
+        for (int v4 = 0; v4 < D / 8; ++v4) {
+          reinterpret_cast<uint4*>(dkr)[v4] = make_uint4(0, 0, 0, 0);
+          reinterpret_cast<uint4*>(dvr)[v4] = make_uint4(0, 0, 0, 0);
+        }
+      }
+    }
+    if (n_steps > 0 && ok && wait_warp(dkv_full, 0)) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const float mul = which == 0 ? args.scale : 1.0f;
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(which == 0 ? args.dk : args.dv) +
+                             ((size_t(b) * args.Nkv + (key_ok ? key : 0)) * args.Hkv + g) * D;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(lane_addr + (which == 0 ? DK_COL : DV_COL) + cc * 32, o);
+          tmem_ld_wait();
+          tmem_reg_fence32(o);
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * mul, __uint_as_float(o[2 * i + 1]) * mul);
+          if (key_ok) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) d4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// D_i = sum_e dO_ie O_ie and LSE'_i = LSE_i * log2 e (+inf when the row has no key), per (b, h) row of
+// whole tiles (padding rows: +inf and 0).
+__global__ void __launch_bounds__(128)
+    attn_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                        const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ dd, int Nq,
+                        int Hq, int Nq_pad) {
+  const int bh = blockIdx.y, b = bh / Hq, h = bh % Hq;
+  const int i = blockIdx.x * 128 + threadIdx.x;
+  if (i >= Nq_pad) return;
+  float l2 = INFINITY, dsum = 0.f;
+  if (i < Nq) {
+    const float L = lse[size_t(bh) * Nq + i];
+    l2 = (L == -INFINITY) ? INFINITY : L * 1.4426950408889634f;
+    const uint4* po = reinterpret_cast<const uint4*>(o + ((size_t(b) * Nq + i) * Hq + h) * bwd::D);
+    const uint4* pd = reinterpret_cast<const uint4*>(dout + ((size_t(b) * Nq + i) * Hq + h) * bwd::D);
+#pragma unroll 4
+    for (int u = 0; u < bwd::D / 8; ++u) {
+      const uint4 a = po[u], c = pd[u];
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wc[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        dsum = fmaf(__uint_as_float(wa[k] << 16), __uint_as_float(wc[k] << 16), dsum);
+        dsum = fmaf(__uint_as_float(wa[k] & 0xFFFF0000u), __uint_as_float(wc[k] & 0xFFFF0000u), dsum);
+      }
+    }
+  }
+  lse2[size_t(bh) * Nq_pad + i] = l2;
+  dd[size_t(bh) * Nq_pad + i] = dsum;
+}
+
+// dQ = scale * accumulator, bf16
+__global__ void attn_bwd_post_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq, size_t n4,
+                                     float scale) {
+  for (size_t i = blockIdx.x * size_t(blockDim.x) + threadIdx.x; i < n4; i += size_t(gridDim.x) * blockDim.x) {
+    const float4 v = reinterpret_cast<const float4*>(acc)[i];
+    uint2 w;
+    w.x = pack_bf16x2(v.x * scale, v.y * scale);
+    w.y = pack_bf16x2(v.z * scale, v.w * scale);
+    reinterpret_cast<uint2*>(dq)[i] = w;
+  }
+}
+
+size_t bwd_workspace(int B, int Hq, int Nq, int d) {
+  const size_t nq_pad = (size_t(Nq) + 127) / 128 * 128;
+  const size_t acc = size_t(B) * Nq * Hq * d * sizeof(float);
+  return ((acc + 255) / 256) * 256 + 2 * size_t(B) * Hq * nq_pad * sizeof(float);
+}
+
+attn_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                           const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nkv,
+                           float scale, int causal, void* workspace, cudaStream_t stream) {
+  using namespace bwd;
+  const int Nq_pad = (Nq + 127) / 128 * 128;
+  const size_t acc_bytes = size_t(B) * Nq * Hq * D * sizeof(float);
+  float* acc = static_cast<float*>(workspace);
+  float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + ((acc_bytes + 255) / 256) * 256);
+  float* dd = lse2 + size_t(B) * Hq * Nq_pad;
+  CUtensorMap tmQ, tmK, tmV, tmDO;
+  if (!encode_tile_map(&tmQ, q, D, Hq, Nq, B, 64, BM, 128) || !encode_tile_map(&tmK, k, D, Hkv, Nkv, B, 64, BN, 128) ||
+      !encode_tile_map(&tmV, v, D, Hkv, Nkv, B, 64, BN, 128) ||
+      !encode_tile_map(&tmDO, dout, D, Hq, Nq, B, 64, BM, 128))
+    return ATTN_ERR_CUDA;
+  if (ensure_dyn_smem(reinterpret_cast<const void*>(attn_bwd_kernel), SMEM_BYTES) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemsetAsync(acc, 0, acc_bytes, stream) != cudaSuccess) return ATTN_ERR_CUDA;
+  attn_bwd_pre_kernel<<<dim3(Nq_pad / 128, B * Hq), 128, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dout), lse, lse2, dd, Nq, Hq,
+      Nq_pad);
+  BwdArgs a;
+  a.dk = dk;
+  a.dv = dv;
+  a.dq_acc = acc;
+  a.lse2 = lse2;
+  a.dd = dd;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Nq = Nq;
+  a.Nkv = Nkv;
+  a.Nq_pad = Nq_pad;
+  a.group = Hq / Hkv;
+  a.n_kb = (Nkv + BN - 1) / BN;
+  a.causal = causal;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.scale = scale;
+  a.timeout_ns = kWaitLimitNs;
+  const long long grid = (long long)a.n_kb * B * Hkv;
+  if (grid > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
+  attn_bwd_kernel<<<dim3(unsigned(grid)), THREADS, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmDO, a);
+  const size_t n4 = size_t(B) * Nq * Hq * D / 4;
+  attn_bwd_post_kernel<<<dim3(unsigned(n4 / 256 + 1 < 8192 ? n4 / 256 + 1 : 8192)), 256, 0, stream>>>(
+      acc, reinterpret_cast<__nv_bfloat16*>(dq), n4, scale);
+  return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
+}
+
+}  // namespace attn

@@ -76,6 +76,11 @@ attn_status_t fwd_fp8_dispatch(const void* q8, const void* k8, const void* vt8, 
 attn_status_t fp8_quantize_dispatch(const void* x, const float* signs, void* codes, float* amax, int B, int N, int H,
                                     int transpose, cudaStream_t stream);
 
+size_t bwd_workspace(int B, int Hq, int Nq, int d);
+attn_status_t bwd_dispatch(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                           const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nkv,
+                           float scale, int causal, void* workspace, cudaStream_t stream);
+
 int decode_default_chunk(int B, int Hkv, int Nkv_cap);
 size_t decode_workspace(int B, int Hq, int d, int Nkv_cap, int chunk);
 attn_status_t decode_split_dispatch(const void* q, const void* kc, const void* vc, const int32_t* lens, int cap,

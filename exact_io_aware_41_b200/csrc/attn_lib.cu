@@ -6,3 +6,4 @@
 #include "attn_decode.cu"
 #include "attn_decode_static.cu"
 #include "attn_fp8.cu"
+#include "attn_bwd.cu"

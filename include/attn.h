@@ -104,6 +104,26 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, cons
                            float scale, int causal, cudaStream_t stream);
 
 /*
+ * Backward pass: the gradients of a scalar loss L through O = softmax(scale * Q K^T) V, given
+ * dO = dL/dO, recomputing S tile by tile instead of storing it (FlashAttention generation
+ * comparison record, "Workarounds": recompute S in backward). With P = exp(scale * S - LSE):
+ *   dV = P^T dO,  dP = dO V^T,  D = rowsum(dO * O),  dS = P * (dP - D),
+ *   dQ = scale * dS K,  dK = scale * dS^T Q  (dK, dV summed over the query heads of a GQA group).
+ * Products on the tensor cores in bf16 with fp32 accumulation; P and dS are rounded to bf16 before
+ * the products that take them; dQ is accumulated in fp32 in the workspace.
+ *   q, o, dout  bf16 [B, Nq, Hq, d];  k, v bf16 [B, Nkv, Hkv, d];  lse fp32 [B, Hq, Nq] (from
+ *               attn_fwd with the same q, k, v, scale and causal flag), all read only
+ *   dq          bf16 [B, Nq, Hq, d];  dk, dv bf16 [B, Nkv, Hkv, d], written
+ *   workspace   caller-owned, at least attn_bwd_workspace_bytes(B, Hq, Nq, d) bytes, 256-byte
+ *               aligned, no initialisation needed (the call zeroes what it accumulates into)
+ *   d = 128 (ATTN_ERR_UNSUPPORTED otherwise); B * Hq <= 65535; everything else as attn_fwd.
+ */
+size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq, int d);
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                       void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq, int Nkv, int d, float scale,
+                       int causal, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Bytes of device workspace attn_decode_splitkv needs: the per-split partial outputs
  * (fp32 [B, Hq, n_splits, d]) and partial LSEs (fp32 [B, Hq, n_splits]), n_splits =
  * ceil(Nkv_cap / chunk). chunk = 0 selects the same automatic chunk attn_decode_splitkv uses.
@@ -196,7 +216,7 @@ const char* attn_status_string(attn_status_t status);
 
 /*
  * Name of the kernel(s) that `which` selects (0 = prefill forward, bf16 or 8-bit, 1 = decode split,
- * 2 = decode combine), for recording which kernel a measurement ran (the evolution article's section 1.1
+ * 2 = decode combine, 3 = backward), for recording which kernel a measurement ran (the evolution article's section 1.1
  * asks that a benchmark name its kernel). Returns NULL for an unknown index.
  */
 const char* attn_kernel_name(int which);

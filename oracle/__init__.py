@@ -314,3 +314,37 @@ def fp8_quantize(x, signs=None):
 def fp8_dequantize(codes, amax) -> np.ndarray:
     """Values the codes stand for: code value * amax / 448 per (batch, head), fp64; [B, N, H, d]."""
     return e4m3_decode(codes) * (np.asarray(amax, dtype=np.float64) / E4M3_MAX)[:, None, :, None]
+
+
+# ------------------------------------------------------------------------------------------------
+# Backward pass. The FlashAttention generation comparison record ("Workarounds", FA-1) recomputes S
+# in the backward pass instead of storing it; what the pass computes is the gradient of the exact
+# forward above. With L a scalar loss and dO = dL/dO, per (batch, query head), materialised in fp64:
+#   P = softmax(scale * Q K^T) (visible keys),  dV = P^T dO,  dP = dO V^T,
+#   D_i = sum_j P_ij dP_ij,  dS = P * (dP - D),  dQ = scale * dS K,  dK = scale * dS^T Q,
+# and dK, dV of a kv head are the sums over the query heads that read it (GQA).
+# ------------------------------------------------------------------------------------------------
+
+def attention_backward(q, k, v, do, scale: float, causal: bool):
+    """Gradients (dQ [B, Nq, Hq, d], dK, dV [B, Nkv, Hkv, d]) of sum(O * dO) for O = attention(...)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    B, Nq, Hq, d = q.shape
+    _, Nkv, Hkv, _ = k.shape
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for hq in range(Hq):
+            g = kv_head(hq, Hq, Hkv)
+            P = probabilities(q[b, :, hq], k[b, :, g], scale, causal)
+            dO = do[b, :, hq]
+            dv[b, :, g] += P.T @ dO
+            dP = dO @ v[b, :, g].T
+            Dd = (P * dP).sum(axis=1, keepdims=True)
+            dS = P * (dP - Dd)
+            dq[b, :, hq] = scale * (dS @ k[b, :, g])
+            dk[b, :, g] += scale * (dS.T @ q[b, :, hq])
+    return dq, dk, dv

@@ -151,3 +151,23 @@ def assert_parity_fp8(o_gpu, lse_gpu, o_ref, lse_ref, sigma, what):
     if (~ref_inf).any():
         l_err = np.abs(lse_gpu[~ref_inf] - lse_ref[~ref_inf])
         assert l_err.max() <= LSE_ABS, f"{what}: LSE max-abs {l_err.max():.3e}"
+
+
+# Backward pass: each gradient element is a sum of products in which one factor (P for dV; dS for dQ
+# and dK) was rounded to bf16 (relative 2^-9), D comes from the bf16 O, and the result is rounded to
+# bf16 (2^-9). The error of a tensor is therefore a small multiple of 2^-9 of its own magnitude. Gate:
+# RMS error <= 2^-7 x RMS of the reference, and every element within 2^-5 x max |reference|.
+BWD_RMS_REL = 2.0 ** -7
+BWD_MAX_REL = 2.0 ** -5
+
+
+def assert_grad_parity(g_gpu, g_ref, what):
+    assert g_gpu.shape == g_ref.shape, what
+    assert np.all(np.isfinite(g_gpu)), f"{what}: non-finite"
+    err = g_gpu - g_ref
+    rms_ref = np.sqrt(np.mean(g_ref ** 2))
+    rms_err = np.sqrt(np.mean(err ** 2))
+    max_ref = np.abs(g_ref).max()
+    assert rms_err <= BWD_RMS_REL * rms_ref + 1e-7, f"{what}: RMS error {rms_err:.3e} vs RMS {rms_ref:.3e}"
+    assert np.abs(err).max() <= BWD_MAX_REL * max_ref + 1e-6, \
+        f"{what}: max error {np.abs(err).max():.3e} vs max {max_ref:.3e} (RMS error {rms_err:.3e} / {rms_ref:.3e})"
