@@ -10,13 +10,18 @@
 //   S^T = K Q^T      (M = keys, N = queries)           -> TMEM columns [0, 128)
 //   dP^T = V dO^T                                      -> TMEM columns [128, 256)
 //   softmax warps (thread = key row): P^T = exp2(S^T * scale * log2 e - LSE * log2 e), masked;
-//   dS^T = P^T * (dP^T - D); P^T (bf16) over S^T, dS^T (bf16) over dP^T and into shared memory
+//   dS^T = P^T * (dP^T - D); P^T (bf16) over S^T, dS^T (bf16) over dP^T (each 32-query chunk's
+//   16 packed columns at the start of its own 32 score columns) and dS^T into shared memory
 //   dV += P^T dO     (A = P^T in TMEM, B = dO read MN-major)   -> columns [256, 384), whole unit
 //   dK += dS^T Q     (A = dS^T in TMEM, B = Q read MN-major)   -> columns [384, 512), whole unit
-//   dQ  = dS K       (A = dS from shared memory, M-major; B = K read MN-major) -> columns [0, 128)
-//   the same warps add dQ (thread = query row) into an fp32 accumulator with vector atomics.
-// MMAs issued by one thread execute in issue order, so dQ may overwrite P^T's columns after the dV
-// product that reads them. The unit ends with dK (times scale) and dV stored as bf16.
+//   dQ  = dS K       (A = dS from shared memory, M-major; B = K read MN-major) -> columns [128, 256)
+//   the same warps stage dQ (thread = query row) in the step's Q / dO buffer, and the TMA unit adds
+//   it into an fp32 accumulator (cp.reduce.async.bulk.tensor ... add).
+// MMAs issued by one thread execute in issue order, so dQ may overwrite dS^T's columns after the dK
+// product that reads them, and the next step's S^T may overwrite P^T's after the dV product. Eight
+// warps (two per TMEM lane quadrant, 64 of the 128 columns each) do the elementwise work; Q, dO and
+// their LSE' and D rows are double-buffered so the next step's loads overlap this one. The unit ends
+// with dK (times scale) and dV stored as bf16.
 //
 // A pre-pass writes D and LSE * log2 e per query row (padded to whole tiles; rows without keys or
 // past Nq get LSE' = +inf, so their P is 0) and zeroes the dQ accumulator; a post-pass rounds
@@ -35,14 +40,23 @@ constexpr int BM = 128;                       // query rows per step
 constexpr int BN = 128;                       // keys per CTA
 constexpr int CHUNK_BYTES = 128 * 128;        // 64-column chunk of a 128-row tile (128-byte rows)
 constexpr int TILE_BYTES = 2 * CHUNK_BYTES;   // 128 x 128 bf16
-constexpr int THREADS = 256;
+constexpr int NSW = 8;                        // softmax / epilogue warps: two per TMEM lane quadrant
+constexpr int THREADS = 128 + 32 * NSW;
 constexpr int TMEM_COLS = 512;
 constexpr int S_COL = 0, DP_COL = 128, DV_COL = 256, DK_COL = 384;
-// shared memory: K, V, Q, dO, dS tiles, LSE' and D rows, barriers
-constexpr int OFF_K = 0, OFF_V = TILE_BYTES, OFF_Q = 2 * TILE_BYTES, OFF_DO = 3 * TILE_BYTES, OFF_DS = 4 * TILE_BYTES;
-constexpr int OFF_LSE = 5 * TILE_BYTES, OFF_DD = OFF_LSE + BM * 4, OFF_BAR = OFF_DD + BM * 4;
-constexpr int NBARS = 8;  // kv_full, q_full, q_empty, s_full, p_full, dq_full, dq_free, dkv_full
-constexpr int SMEM_BYTES = 1024 + OFF_BAR + NBARS * 8 + 16;
+// shared memory (tiles first, 1024-byte aligned): K, V, dS, then Q and dO of two stages; then the
+// two stages' LSE' and D rows and the barriers. The whole budget (about 226 KB) leaves no room to
+// pad for alignment, so the kernel checks that its dynamic shared memory starts on a 1024-byte
+// boundary (it does when the kernel declares no static shared memory) and otherwise records an
+// error and does nothing.
+constexpr int OFF_K = 0, OFF_V = TILE_BYTES, OFF_DS = 2 * TILE_BYTES;
+constexpr int OFF_Q0 = 3 * TILE_BYTES;        // stage s: Q at OFF_Q0 + 2s tiles, dO right after it
+constexpr int OFF_LSE0 = 7 * TILE_BYTES;      // stage s: LSE' at OFF_LSE0 + s * 1024, D 512 bytes later
+constexpr int OFF_BAR = OFF_LSE0 + 2 * 1024;
+// kv_full, q_full[2], q_empty[2], s_full, p_full, dq_full, dq_free, dkv_full
+constexpr int NBARS = 10;
+constexpr int SMEM_BYTES = OFF_BAR + NBARS * 8 + 16;
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 }  // namespace bwd
 
 struct BwdArgs {
@@ -65,9 +79,22 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
                : "memory");
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
+// Adds a shared-memory box into global memory through the TMA unit (element-wise fp32 add at the
+// destination), tracked by the issuing thread's bulk async-group.
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const void* smem_src, int c0, int c1, int c2,
+                                                  int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until every bulk copy of this thread's committed groups has completed (writes performed).
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Waits until every bulk copy of this thread's committed groups has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
 // First query tile whose rows see some key of block kb (causal: key j visible to row i iff
@@ -81,23 +108,24 @@ __device__ __forceinline__ int first_q_tile(const BwdArgs& a, int kb) {
 __global__ void __launch_bounds__(bwd::THREADS, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const BwdArgs args) {
+                    const __grid_constant__ CUtensorMap tmDQ, const BwdArgs args) {
   using namespace bwd;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicOr(&g_error_word, kErrSmemAlignBit);
+    return;  // every thread of the CTA takes this branch: nothing was started
+  }
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;
-  uint64_t* q_empty = bars + 2;
-  uint64_t* s_full = bars + 3;
-  uint64_t* p_full = bars + 4;
-  uint64_t* dq_full = bars + 5;
-  uint64_t* dq_free = bars + 6;
-  uint64_t* dkv_full = bars + 7;
+  uint64_t* q_full = bars + 1;   // [2]
+  uint64_t* q_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* p_full = bars + 6;
+  uint64_t* dq_full = bars + 7;
+  uint64_t* dq_free = bars + 8;
+  uint64_t* dkv_full = bars + 9;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  const float* s_lse = reinterpret_cast<const float*>(smem + OFF_LSE);
-  const float* s_dd = reinterpret_cast<const float*>(smem + OFF_DD);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint64_t T = args.timeout_ns;
@@ -112,7 +140,16 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
   const int n_steps = steps_per_head * args.group;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NBARS; ++i) mbar_init(&bars[i], (i == 4 || i == 6) ? 4 : 1);  // p_full, dq_free: 4 warps
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], NSW);  // the softmax warps release a stage (its space stages dQ last)
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, NSW);   // one arrival per softmax warp
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, NSW);  // one arrival per softmax warp
+    mbar_init(dkv_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -124,19 +161,6 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-
-  // descriptors: K-major tiles (rows of d) and MN-major reads of the same tiles
-  const uint64_t dK_k = smem_desc(smem_u32(smem + OFF_K), 16, 1024, kLayoutSW128);
-  const uint64_t dV_k = smem_desc(smem_u32(smem + OFF_V), 16, 1024, kLayoutSW128);
-  const uint64_t dQ_k = smem_desc(smem_u32(smem + OFF_Q), 16, 1024, kLayoutSW128);
-  const uint64_t dDO_k = smem_desc(smem_u32(smem + OFF_DO), 16, 1024, kLayoutSW128);
-  const uint64_t dQ_mn = smem_desc(smem_u32(smem + OFF_Q), CHUNK_BYTES, 1024, kLayoutSW128);
-  const uint64_t dDO_mn = smem_desc(smem_u32(smem + OFF_DO), CHUNK_BYTES, 1024, kLayoutSW128);
-  const uint64_t dK_mn = smem_desc(smem_u32(smem + OFF_K), CHUNK_BYTES, 1024, kLayoutSW128);
-  const uint64_t dDS_mn = smem_desc(smem_u32(smem + OFF_DS), CHUNK_BYTES, 1024, kLayoutSW128);
-  constexpr uint32_t idesc_kk = idesc_bf16_f32(128, 128, 0, 0);   // A, B K-major
-  constexpr uint32_t idesc_tmn = idesc_bf16_f32(128, 128, 0, 1);  // A from TMEM, B MN-major
-  constexpr uint32_t idesc_mnmn = idesc_bf16_f32(128, 128, 1, 1); // A, B MN-major
 
   auto step_coords = [&](int t, int& h, int& qt) {
     h = g * args.group + t / steps_per_head;
@@ -157,36 +181,61 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
       }
       int t = 0;
       for (; t < n_steps; ++t) {
-        if (t > 0 && !mbar_wait(q_empty, uint32_t((t - 1) & 1), abort_flag, T)) break;
+        const int st = t & 1;
+        // the stage's previous contents (step t - 2) are no longer read by any MMA
+        if (t >= 2 && !mbar_wait(&q_empty[st], uint32_t(((t - 2) >> 1) & 1), abort_flag, T)) break;
         int h, qt;
         step_coords(t, h, qt);
-        mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES + 2 * BM * 4);
+        uint8_t* sq = smem + OFF_Q0 + 2 * st * TILE_BYTES;
+        mbar_arrive_expect_tx(&q_full[st], 2 * TILE_BYTES + 2 * BM * 4);
         for (int c = 0; c < 2; ++c) {
-          tma_load_4d(smem + OFF_Q + c * CHUNK_BYTES, &tmQ, q_full, c * 64, h, qt * BM, b);
-          tma_load_4d(smem + OFF_DO + c * CHUNK_BYTES, &tmDO, q_full, c * 64, h, qt * BM, b);
+          tma_load_4d(sq + c * CHUNK_BYTES, &tmQ, &q_full[st], c * 64, h, qt * BM, b);
+          tma_load_4d(sq + TILE_BYTES + c * CHUNK_BYTES, &tmDO, &q_full[st], c * 64, h, qt * BM, b);
         }
         const size_t row = size_t(b * args.Hq + h) * args.Nq_pad + size_t(qt) * BM;
-        bulk_load(smem + OFF_LSE, args.lse2 + row, BM * 4, q_full);
-        bulk_load(smem + OFF_DD, args.dd + row, BM * 4, q_full);
+        bulk_load(smem + OFF_LSE0 + st * 1024, args.lse2 + row, BM * 4, &q_full[st]);
+        bulk_load(smem + OFF_LSE0 + st * 1024 + 512, args.dd + row, BM * 4, &q_full[st]);
       }
       // copies in flight land before the CTA exits (bounded)
       mbar_wait(kv_full, 0, nullptr, 100000000ull);
-      if (t > 0) mbar_wait(q_full, uint32_t((t - 1) & 1), nullptr, 100000000ull);
+      for (int u = t - 2; u < t; ++u)
+        if (u >= 0) mbar_wait(&q_full[u & 1], uint32_t((u >> 1) & 1), nullptr, 100000000ull);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ================================ MMA issuer ================================
     if (lane == 0 && n_steps > 0) {
+      // K-major reads of K, V, Q, dO (rows of d) and MN-major reads of Q, dO, K and the dS tile
+      const uint64_t dK_k = smem_desc(smem_u32(smem + OFF_K), 16, 1024, kLayoutSW128);
+      const uint64_t dV_k = smem_desc(smem_u32(smem + OFF_V), 16, 1024, kLayoutSW128);
+      const uint64_t dK_mn = smem_desc(smem_u32(smem + OFF_K), CHUNK_BYTES, 1024, kLayoutSW128);
+      const uint64_t dDS_mn = smem_desc(smem_u32(smem + OFF_DS), CHUNK_BYTES, 1024, kLayoutSW128);
+      constexpr uint32_t idesc_kk = idesc_bf16_f32(128, 128, 0, 0);    // A, B K-major
+      constexpr uint32_t idesc_tmn = idesc_bf16_f32(128, 128, 0, 1);   // A from TMEM, B MN-major
+      constexpr uint32_t idesc_mnmn = idesc_bf16_f32(128, 128, 1, 1);  // A, B MN-major
       bool ok = mbar_wait(kv_full, 0, abort_flag, T);
       for (int t = 0; t < n_steps && ok; ++t) {
-        ok = mbar_wait(q_full, uint32_t(t & 1), abort_flag, T);
-        if (ok && t > 0) ok = mbar_wait(dq_free, uint32_t((t - 1) & 1), abort_flag, T);  // columns [0, 128) read
+        const int st = t & 1;
+        const uint32_t sq = smem_u32(smem + OFF_Q0 + 2 * st * TILE_BYTES);
+        const uint64_t dQ_k = smem_desc(sq, 16, 1024, kLayoutSW128);
+        const uint64_t dDO_k = smem_desc(sq + TILE_BYTES, 16, 1024, kLayoutSW128);
+        const uint64_t dQ_mn = smem_desc(sq, CHUNK_BYTES, 1024, kLayoutSW128);
+        const uint64_t dDO_mn = smem_desc(sq + TILE_BYTES, CHUNK_BYTES, 1024, kLayoutSW128);
+        ok = mbar_wait(&q_full[st], uint32_t((t >> 1) & 1), abort_flag, T);
         if (!ok) break;
         tc_fence_after();
+        // S^T = K Q^T into [0, 128): P^T of the previous step there was read by its dV product,
+        // issued earlier by this thread
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * CHUNK_BYTES + (kk % 4) * 32) >> 4;
           umma_ss(tmem + S_COL, dK_k + off, dQ_k + off, idesc_kk, kk > 0 ? 1u : 0u);
+        }
+        // dP^T = V dO^T into [128, 256), once the previous step's dQ (there) has been read out
+        if (t > 0) {
+          ok = mbar_wait(dq_free, uint32_t((t - 1) & 1), abort_flag, T);
+          if (!ok) break;
+          tc_fence_after();
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -197,21 +246,23 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
         ok = mbar_wait(p_full, uint32_t(t & 1), abort_flag, T);
         if (!ok) break;
         tc_fence_after();
-        // over the step's 128 queries (k-steps of 16): dV += P^T dO, dK += dS^T Q, dQ = dS K
+        // over the step's 128 queries (k-steps of 16): dV += P^T dO, dK += dS^T Q, then dQ = dS K
+        // into [128, 256), after the dK product has read dS^T there
+        // A = P^T / dS^T: queries 16kk .. 16kk+15 are columns 8 (kk % 2) .. of chunk kk / 2, which
+        // starts at column 32 (kk / 2)
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ts(tmem + DV_COL, tmem + S_COL + kk * 8, dDO_mn + uint64_t((kk * 16 * 128) >> 4), idesc_tmn,
-                  (t > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + DV_COL, tmem + S_COL + 32 * (kk / 2) + 8 * (kk % 2),
+                  dDO_mn + uint64_t((kk * 16 * 128) >> 4), idesc_tmn, (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
-          umma_ts(tmem + DK_COL, tmem + DP_COL + kk * 8, dQ_mn + uint64_t((kk * 16 * 128) >> 4), idesc_tmn,
-                  (t > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tmem + DK_COL, tmem + DP_COL + 32 * (kk / 2) + 8 * (kk % 2),
+                  dQ_mn + uint64_t((kk * 16 * 128) >> 4), idesc_tmn, (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ss(tmem + S_COL, dDS_mn + uint64_t((kk * 16 * 128) >> 4), dK_mn + uint64_t((kk * 16 * 128) >> 4),
+          umma_ss(tmem + DP_COL, dDS_mn + uint64_t((kk * 16 * 128) >> 4), dK_mn + uint64_t((kk * 16 * 128) >> 4),
                   idesc_mnmn, kk > 0 ? 1u : 0u);
         umma_commit(dq_full);
-        umma_commit(q_empty);
         if (t == n_steps - 1) umma_commit(dkv_full);
       }
       if (!ok) {
@@ -225,7 +276,8 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
   } else if (warp >= 4) {
     // ========================= softmax / dQ / dK dV epilogue warps =========================
     const int wq = warp & 3;
-    const int row = wq * 32 + lane;  // TMEM lane: key row (softmax, dK dV) or query row (dQ)
+    const int hf = (warp - 4) >> 2;   // which 64 of the 128 columns this warp covers
+    const int row = wq * 32 + lane;   // TMEM lane: key row (softmax, dK dV) or query row (dQ)
     const uint32_t lane_addr = tmem + (uint32_t(wq * 32) << 16);
     const float c = args.scale_log2;
     const int key = kb * BN + row;
@@ -238,6 +290,8 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
     for (int t = 0; t < n_steps && ok; ++t) {
       int h, qt;
       step_coords(t, h, qt);
+      const float* s_lse = reinterpret_cast<const float*>(smem + OFF_LSE0 + (t & 1) * 1024);
+      const float* s_dd = s_lse + 128;
       if (!wait_warp(s_full, uint32_t(t & 1))) {
         ok = false;
         break;
@@ -245,32 +299,42 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
       tc_fence_after();
       const int q0 = qt * BM;
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {  // 32 query columns at a time
+      for (int cx = 0; cx < 2; ++cx) {  // 32 query columns at a time, this warp's 64
+        const int cc = 2 * hf + cx;
         uint32_t sv[32], dpv[32];
         tmem_ld32(lane_addr + S_COL + cc * 32, sv);
         tmem_ld32(lane_addr + DP_COL + cc * 32, dpv);
         tmem_ld_wait();
         tmem_reg_fence32(sv);
         tmem_reg_fence32(dpv);
+        // warp-uniform: does some (key, query) of this 32 x 32 block fall outside the mask? (rows
+        // past Nq need no test: their LSE' is +inf, so P = 0)
+        const int qf = q0 + cc * 32;
+        const bool need_mask = (kb * BN + BN > args.Nkv) || (args.causal && kb * BN + BN - 1 > qf + diag);
         uint32_t pk[16], dk2[16];
 #pragma unroll
-        for (int i2 = 0; i2 < 16; ++i2) {
-          float p2[2], ds2[2];
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(s_lse + cc * 32 + 4 * i4);
+          const float4 d4 = *reinterpret_cast<const float4*>(s_dd + cc * 32 + 4 * i4);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+          float p4[4], ds4[4];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int qi = cc * 32 + 2 * i2 + u;
-            const int qrow = q0 + qi;
-            const bool vis = key_ok && (!args.causal || key <= qrow + diag);
-            const float p = vis ? ex2(fmaf(__uint_as_float(sv[2 * i2 + u]), c, -s_lse[qi])) : 0.f;
-            p2[u] = p;
-            ds2[u] = p * (__uint_as_float(dpv[2 * i2 + u]) - s_dd[qi]);
+          for (int u = 0; u < 4; ++u) {
+            const int qi = cc * 32 + 4 * i4 + u;
+            float p = ex2(fmaf(__uint_as_float(sv[4 * i4 + u]), c, -lv[u]));
+            if (need_mask && !(key_ok && (!args.causal || key <= q0 + qi + diag))) p = 0.f;
+            p4[u] = p;
+            ds4[u] = p * (__uint_as_float(dpv[4 * i4 + u]) - dv4[u]);
           }
-          pk[i2] = pack_bf16x2(p2[0], p2[1]);
-          dk2[i2] = pack_bf16x2(ds2[0], ds2[1]);
+          pk[2 * i4] = pack_bf16x2(p4[0], p4[1]);
+          pk[2 * i4 + 1] = pack_bf16x2(p4[2], p4[3]);
+          dk2[2 * i4] = pack_bf16x2(ds4[0], ds4[1]);
+          dk2[2 * i4 + 1] = pack_bf16x2(ds4[2], ds4[3]);
         }
-        // P^T over S^T and dS^T over dP^T (columns already read), both bf16 pairs
-        tmem_st16(lane_addr + S_COL + cc * 16, pk);
-        tmem_st16(lane_addr + DP_COL + cc * 16, dk2);
+        // P^T over S^T and dS^T over dP^T, bf16 pairs: the chunk's 16 columns go to the first 16 of
+        // its own 32 score columns (just read), so no warp writes where the other still reads
+        tmem_st16(lane_addr + S_COL + cc * 32, pk);
+        tmem_st16(lane_addr + DP_COL + cc * 32, dk2);
         // dS^T row into the shared tile [key][query] (128-byte swizzled, 64-query chunks): the A
         // operand of dQ = dS K, read M-major
 #pragma unroll
@@ -289,40 +353,59 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
-      // dQ of this step (thread = query row q0 + row): add into the fp32 accumulator
+      // the previous step's dQ boxes (in that step's Q / dO buffer) have been read by the TMA unit
+      // by now, as a rule: hand the buffer back to the producer for the step after this one
+      if (t > 0 && lane == 0) {
+        bulk_wait_group_read0();
+        mbar_arrive(&q_empty[(t - 1) & 1]);
+      }
+      // dQ of this step (thread = query row q0 + row, this warp's 64 of the d columns): once every
+      // product of the step is done, read it from TMEM and release those columns, then stage it as
+      // two 32 x 32 fp32 boxes (128-byte rows, swizzled like the tensor map) in this step's Q / dO
+      // buffer, which no product reads any more, and let the TMA unit add the boxes into the fp32
+      // accumulator. The buffer goes back to the producer once the TMA has read it (checked one
+      // step later, above).
       if (!wait_warp(dq_full, uint32_t(t & 1))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int qrow = q0 + row;
-      float* dst = args.dq_acc + ((size_t(b) * args.Nq + (qrow < args.Nq ? qrow : 0)) * args.Hq + h) * D;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(lane_addr + S_COL + cc * 32, o);
-        tmem_ld_wait();
-        tmem_reg_fence32(o);
-        if (qrow < args.Nq) {
-#pragma unroll
-          for (int v4 = 0; v4 < 8; ++v4)
-            red_add_v4(dst + cc * 32 + 4 * v4, __uint_as_float(o[4 * v4]), __uint_as_float(o[4 * v4 + 1]),
-                       __uint_as_float(o[4 * v4 + 2]), __uint_as_float(o[4 * v4 + 3]));
-        }
-      }
+      uint32_t o[2][32];
+      tmem_ld32(lane_addr + DP_COL + (2 * hf) * 32, o[0]);
+      tmem_ld32(lane_addr + DP_COL + (2 * hf + 1) * 32, o[1]);
+      tmem_ld_wait();
+      tmem_reg_fence32(o[0]);
+      tmem_reg_fence32(o[1]);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
-    }
-    // dK (times scale) and dV of this key block, bf16
-    if (key_ok) {
-      __nv_bfloat16* dkr = reinterpret_cast<__nv_bfloat16*>(args.dk) + ((size_t(b) * args.Nkv + key) * args.Hkv + g) * D;
-      __nv_bfloat16* dvr = reinterpret_cast<__nv_bfloat16*>(args.dv) + ((size_t(b) * args.Nkv + key) * args.Hkv + g) * D;
-      if (n_steps == 0) {
-        for (int v4 = 0; v4 < D / 8; ++v4) {
-          reinterpret_cast<uint4*>(dkr)[v4] = make_uint4(0, 0, 0, 0);
-          reinterpret_cast<uint4*>(dvr)[v4] = make_uint4(0, 0, 0, 0);
+      const int row0 = q0 + wq * 32;  // first query row of this warp's boxes
+      uint8_t* box = smem + OFF_Q0 + 2 * (t & 1) * TILE_BYTES + (warp - 4) * 8192;
+#pragma unroll
+      for (int cx = 0; cx < 2; ++cx)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t a = smem_u32(box + cx * 4096) + lane * 128 + ((u ^ (lane & 7)) << 4);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(o[cx][4 * u]), "r"(o[cx][4 * u + 1]),
+                       "r"(o[cx][4 * u + 2]), "r"(o[cx][4 * u + 3])
+                       : "memory");
         }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && row0 < args.Nq) {  // rows past Nq are clipped by the TMA unit
+        tma_reduce_add_4d(&tmDQ, box, (2 * hf) * 32, h, row0, b);
+        tma_reduce_add_4d(&tmDQ, box + 4096, (2 * hf + 1) * 32, h, row0, b);
+        bulk_commit_group();
+      }
+      __syncwarp();
+    }
+    if (lane == 0) bulk_wait_group0();  // this warp's dQ additions have been performed
+    // dK (times scale) and dV of this key block, bf16, this warp's 64 of the d columns
+    if (key_ok && n_steps == 0) {
+      for (int which = 0; which < 2; ++which) {
+        uint4* dz = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(which ? args.dv : args.dk) +
+                                             ((size_t(b) * args.Nkv + key) * args.Hkv + g) * D + 64 * hf);
+        for (int v4 = 0; v4 < 8; ++v4) dz[v4] = make_uint4(0, 0, 0, 0);
       }
     }
     if (n_steps > 0 && ok && wait_warp(dkv_full, 0)) {
@@ -333,7 +416,8 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
         __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(which == 0 ? args.dk : args.dv) +
                              ((size_t(b) * args.Nkv + (key_ok ? key : 0)) * args.Hkv + g) * D;
 #pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cx = 0; cx < 2; ++cx) {
+          const int cc = 2 * hf + cx;
           uint32_t o[32];
           tmem_ld32(lane_addr + (which == 0 ? DK_COL : DV_COL) + cc * 32, o);
           tmem_ld_wait();
@@ -422,6 +506,12 @@ attn_status_t bwd_dispatch(const void* q, const void* k, const void* v, const vo
       !encode_tile_map(&tmV, v, D, Hkv, Nkv, B, 64, BN, 128) ||
       !encode_tile_map(&tmDO, dout, D, Hq, Nq, B, 64, BM, 128))
     return ATTN_ERR_CUDA;
+  CUtensorMap tmDQ;
+  {
+    const long long dims[4] = {D, Hq, Nq, B};
+    const int box[4] = {32, 1, 32, 1};
+    if (!encode_map(&tmDQ, acc, 4, dims, box, 128)) return ATTN_ERR_CUDA;
+  }
   if (ensure_dyn_smem(reinterpret_cast<const void*>(attn_bwd_kernel), SMEM_BYTES) != cudaSuccess) return ATTN_ERR_CUDA;
   if (cudaMemsetAsync(acc, 0, acc_bytes, stream) != cudaSuccess) return ATTN_ERR_CUDA;
   attn_bwd_pre_kernel<<<dim3(Nq_pad / 128, B * Hq), 128, 0, stream>>>(
@@ -447,7 +537,7 @@ attn_status_t bwd_dispatch(const void* q, const void* k, const void* v, const vo
   a.timeout_ns = kWaitLimitNs;
   const long long grid = (long long)a.n_kb * B * Hkv;
   if (grid > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
-  attn_bwd_kernel<<<dim3(unsigned(grid)), THREADS, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmDO, a);
+  attn_bwd_kernel<<<dim3(unsigned(grid)), THREADS, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmDO, tmDQ, a);
   const size_t n4 = size_t(B) * Nq * Hq * D / 4;
   attn_bwd_post_kernel<<<dim3(unsigned(n4 / 256 + 1 < 8192 ? n4 / 256 + 1 : 8192)), 256, 0, stream>>>(
       acc, reinterpret_cast<__nv_bfloat16*>(dq), n4, scale);

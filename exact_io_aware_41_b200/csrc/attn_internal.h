@@ -12,6 +12,7 @@ namespace attn {
 // Bits of the device error word (g_error_word).
 enum : unsigned int {
   kErrBadLengthBit = 2u,  // a decode length outside [0, Nkv_cap] was clamped
+  kErrSmemAlignBit = 4u,  // a kernel found its dynamic shared memory off its required alignment
 };
 
 // Wall-time limit of every pipeline wait inside a kernel. Far above any legitimate wait (a whole
@@ -50,7 +51,7 @@ int sm_count();
 bool encode_tile_map(CUtensorMap* map, const void* base, int d, int heads, int rows, int outer, int box_cols,
                      int box_rows, unsigned swizzle_bytes);
 
-// The general form: a 4-d tensor of elem_bytes-sized elements (1: 8-bit codes, 2: bf16) with dense
+// The general form: a 4-d tensor of elem_bytes-sized elements (1: 8-bit codes, 2: bf16, 4: fp32) with dense
 // strides, dims[0] innermost, box[] elements per dimension; cached like encode_tile_map.
 bool encode_map(CUtensorMap* map, const void* base, int elem_bytes, const long long* dims, const int* box,
                 unsigned swizzle_bytes);

@@ -207,7 +207,7 @@ attn_status_t attn_decode_combine(const float* part_o, const float* part_lse, in
  * Reads and clears the device error word (synchronises the calling thread with the device).
  * ATTN_OK if no kernel recorded a fault since the last call, ATTN_ERR_TIMEOUT if a bounded
  * pipeline wait gave up, ATTN_ERR_INVALID_ARG if a decode length was out of range, ATTN_ERR_CUDA
- * if the word could not be read.
+ * if the word could not be read or a kernel found its shared memory misaligned (and did nothing).
  */
 attn_status_t attn_get_last_error(void);
 
