@@ -173,6 +173,47 @@ int sm_count() {
   return n;
 }
 
+namespace {
+// per device: the kernel the pair count was taken for, and the count
+struct PairEntry {
+  std::atomic<const void*> func{nullptr};
+  std::atomic<int> pairs{0};
+};
+PairEntry g_pairs[kMaxDevices];
+}  // namespace
+
+int max_pairs(const void* func, int threads, int smem_bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  const bool cacheable = dev >= 0 && dev < kMaxDevices;
+  if (cacheable && g_pairs[dev].func.load(std::memory_order_acquire) == func) {
+    const int cached = g_pairs[dev].pairs.load(std::memory_order_relaxed);
+    if (cached > 0) return cached;
+  }
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  lc.gridDim = dim3(2);
+  lc.blockDim = dim3(threads);
+  lc.dynamicSmemBytes = smem_bytes;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, func, &lc) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  if (n <= 0) return -1;
+  if (cacheable) {
+    g_pairs[dev].pairs.store(n, std::memory_order_relaxed);
+    g_pairs[dev].func.store(func, std::memory_order_release);
+  }
+  return n;
+}
+
 bool is_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace attn

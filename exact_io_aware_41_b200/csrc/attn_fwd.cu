@@ -20,8 +20,10 @@
 //                 normalisation, section 3) and writes O and LSE.
 // With two query tiles per CTA (d <= 128) the two softmax warpgroups alternate with the tensor
 // core: while one tile's softmax runs, the other tile's MMAs run ("overlaps multiple query tiles",
-// section 5). With d = 256 one query tile alternates between two S buffers instead, and its Q tile
-// is copied into TMEM once per unit so the QK MMAs read only K from shared memory.
+// section 5). With d = 256 the O accumulator takes half of tensor memory, so each CTA holds one
+// query tile, which alternates between two S buffers instead; two CTAs form a pair (a cluster of
+// two) that runs 2-SM MMAs (M = 256) over 256 query rows, each CTA loading half of every K/V tile
+// (the evolution article's 2-CTA MMA, section 5).
 //
 // S and P never leave the SM: S is fp32 in TMEM, P is bf16 in TMEM, read by the MMA straight from
 // there. At d = 128 and 256 P is written in place over S, so the next S = Q K^T into that slot
@@ -67,13 +69,21 @@ constexpr float kRescaleTau = 8.0f;
 
 // F8: Q and K are e4m3 codes (rotated), V is given transposed (e4m3 [d, keys] per head), and the
 // products run as kind::f8f6f4 MMAs with 32-element k-steps; P is packed four e4m3 per TMEM column.
-template <int D, bool F8 = false>
+// PAIR (d = 256): a cluster of two CTAs works on 256 query rows, 128 per CTA, with 2-SM MMAs
+// (cta_group::2, M = 256). Each CTA holds half of every K tile (its 64 of the tile's 128 keys) and
+// half of every V tile (its 128 of the d columns), so 128-key tiles fit a 5-stage ring and the QK
+// products run at N = 128 (a 64-key N = 64 product costs ~52 cycles per k-step against 32 for its
+// FLOPs; N = 128 runs at the full rate).
+template <int D, bool F8 = false, bool PAIR = false>
 struct FwdCfg {
   static_assert(!F8 || D == 128, "the 8-bit path is built for d = 128");
+  static_assert(PAIR == (D == 256), "d = 256 runs on CTA pairs, d <= 128 on single CTAs");
   static constexpr int EB = F8 ? 1 : 2;                 // bytes per element of Q, K, V
   static constexpr int BM = 128;                        // query rows per tile (TMEM lanes)
   static constexpr int NQT = (D <= 128) ? 2 : 1;        // query tiles per CTA
-  static constexpr int BN = (D <= 128) ? 128 : 64;      // keys per K/V tile
+  static constexpr int BN = (D <= 128 || PAIR) ? 128 : 64;  // keys per K/V tile
+  static constexpr int CTAS = PAIR ? 2 : 1;             // CTAs per unit
+  static constexpr int UNIT_ROWS = NQT * BM * CTAS;     // query rows per unit
   // d <= 64: P lives in tensor-memory buffers of its own instead of over S, so a tile's next
   // S = Q K^T is computed while the softmax still works on the current one (the two O accumulators
   // leave room for the buffers). d = 128 has no room for them and writes P over S.
@@ -85,11 +95,15 @@ struct FwdCfg {
   static constexpr int KSTEP = 32 / EB;                 // elements per MMA k-step (32 bytes)
   static constexpr int KPC = CHUNK / KSTEP;             // MMA k-steps per chunk
   static constexpr int Q_CHUNK_BYTES = BM * ROWB;
-  static constexpr int KV_CHUNK_BYTES = BN * ROWB;
+  static constexpr int K_ROWS = BN / CTAS;              // keys of a K tile held by one CTA
+  static constexpr int V_COLS = D / CTAS;               // d columns of a V tile held by one CTA
+  static constexpr int K_CHUNK_BYTES = K_ROWS * ROWB;   // one swizzle chunk (CHUNK of d) of the K part
+  static constexpr int V_CHUNK_BYTES = BN * ROWB;       // one swizzle chunk of the V part (all BN keys)
   static constexpr int Q_TILE_BYTES = BM * D * EB;
-  static constexpr int KV_TILE_BYTES = BN * D * EB;
+  static constexpr int KV_TILE_BYTES = BN * D * EB / CTAS;  // one ring stage: this CTA's K or V part
   static_assert(!F8 || BN * EB == 128, "a transposed V tile row (BN keys) is one 128-byte swizzled row");
   static constexpr int STAGES = (D == 256) ? 5 : (KV_TILE_BYTES >= 32768) ? 4 : 8;
+  static constexpr int P_ARRIVALS = 4 * CTAS;           // p_full: one arrival per softmax warp of the unit
   static constexpr int NSMWG = (NQT == 2) ? 2 : 1;      // softmax warpgroups
   static constexpr int THREADS = 128 * (1 + NSMWG);
   // register split (setmaxnreg) with two softmax warpgroups: control warpgroup, softmax warpgroups;
@@ -111,14 +125,8 @@ struct FwdCfg {
   // separate P buffers (bf16 pairs: BN / 2 columns each), after the O accumulators
   static constexpr int P_COL0 = 2 * BN + NQT * D;
   static constexpr int P_COL1 = P_COL0 + BN / 2;
-  // d = 256: the Q tile is copied into TMEM (bf16 pairs, D / 2 columns) once per unit and QK reads
-  // it from there, so the 64-key QK MMAs read only K from shared memory (with Q from shared memory
-  // as well they are shared-memory bound at N = 64)
-  static constexpr bool Q_TMEM = (D == 256);
-  static constexpr int Q_COL = 2 * BN + NQT * D;
   static constexpr int TMEM_COLS = 512;
-  static_assert(2 * BN + NQT * D + (SEP_P ? NQT * BN / 2 : 0) + (Q_TMEM ? D / 2 : 0) <= TMEM_COLS,
-                "tensor memory budget");
+  static_assert(2 * BN + NQT * D + (SEP_P ? NQT * BN / 2 : 0) <= TMEM_COLS, "tensor memory budget");
   // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done, o_final[2], drain,
   // s_free[2], p_free[2], sched_full[SCHED], sched_empty[SCHED]
   static constexpr int SCHED = 4;  // units the producer may claim ahead of the consumers
@@ -157,9 +165,9 @@ struct Unit {
   int n_tile0;   // K/V tiles the first query tile needs (fewer when the last one is above its diagonal)
 };
 
-template <int D>
+template <int D, bool PAIR>
 __device__ __forceinline__ Unit unit_at(const FwdArgs& a, int lin) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, false, PAIR>;
   const int BH = a.B * a.Hq;
   const int per_group = a.heads_per_group * a.n_qblk;
   const int grp = lin / per_group;
@@ -170,10 +178,10 @@ __device__ __forceinline__ Unit unit_at(const FwdArgs& a, int lin) {
   Unit u;
   u.b = bh / a.Hq;
   u.h = bh % a.Hq;
-  u.q0 = qblk * C::NQT * C::BM;
+  u.q0 = qblk * C::UNIT_ROWS;
   int kv_end = a.Nkv;
   if (a.causal) {
-    const int q_last = min(u.q0 + C::NQT * C::BM, a.Nq) - 1;
+    const int q_last = min(u.q0 + C::UNIT_ROWS, a.Nq) - 1;
     kv_end = min(a.Nkv, q_last + (a.Nkv - a.Nq) + 1);
   }
   u.n_tiles = kv_end > 0 ? (kv_end + C::BN - 1) / C::BN : 0;
@@ -185,11 +193,11 @@ __device__ __forceinline__ Unit unit_at(const FwdArgs& a, int lin) {
   return u;
 }
 
-template <int D, bool F8>
-__global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
+template <int D, bool F8, bool PAIR>
+__global__ void __launch_bounds__(FwdCfg<D, F8, PAIR>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdArgs args) {
-  using C = FwdCfg<D, F8>;
+  using C = FwdCfg<D, F8, PAIR>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
@@ -217,6 +225,9 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
   const uint64_t T = args.timeout_ns;
   const int total_units = args.B * args.Hq * args.n_qblk;
   const int diag = args.Nkv - args.Nq;  // key j visible to query i iff j <= i + diag
+  // CTA pair: rank 0 (the leader) issues the MMAs of both; barriers that the MMAs, the TMA copies
+  // of both CTAs or the softmax warps of both CTAs feed live in the leader's shared memory
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
 
   // ---- set-up --------------------------------------------------------------------------------
   if (threadIdx.x == 0) {
@@ -228,7 +239,7 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);  // one arrival per softmax warp
+      mbar_init(&p_full[i], C::P_ARRIVALS);  // one arrival per softmax warp (of both CTAs of a pair)
       mbar_init(&o_final[i], 1);
       mbar_init(&s_free[i], 4);  // one arrival per softmax warp of the tile
       mbar_init(&p_free[i], 1);
@@ -248,11 +259,18 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
     prefetch_tensormap(&tmV);
   }
   if (warp == 2) {
-    tmem_alloc(tmem_holder, C::TMEM_COLS);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_holder, C::TMEM_COLS);  // the same columns in both CTAs
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  // a pair: the peer's barriers are initialised before any remote arrival or copy can reach them
+  if (PAIR) cluster_sync();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   // With two softmax warpgroups the 128 control threads give registers to the 256 softmax threads:
@@ -262,15 +280,17 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
 
   // ---- MMA issue helpers ------------------------------------------------------------------------
   // bf16: V is read MN-major (rows of d); 8-bit: V is given transposed and read K-major like K
-  constexpr uint32_t idesc_qk = F8 ? idesc_e4m3_f32(128, C::BN, 0, 0) : idesc_bf16_f32(128, C::BN, 0, 0);
-  constexpr uint32_t idesc_pv = F8 ? idesc_e4m3_f32(128, D, 0, 0) : idesc_bf16_f32(128, D, 0, 1);
+  // (a pair's MMAs have M = 256: 128 rows in each CTA; each CTA's shared memory holds half of B's N)
+  constexpr int MMA_M = 128 * C::CTAS;
+  constexpr uint32_t idesc_qk = F8 ? idesc_e4m3_f32(128, C::BN, 0, 0) : idesc_bf16_f32(MMA_M, C::BN, 0, 0);
+  constexpr uint32_t idesc_pv = F8 ? idesc_e4m3_f32(128, D, 0, 0) : idesc_bf16_f32(MMA_M, D, 0, 1);
   // Only the start-address field (bits 0-13, 16-byte units) differs between the descriptors of one
   // operand, so each base descriptor is built once and the k-step offsets are added to it.
   // Shared-memory addresses stay below 2^18, so the field never carries into its neighbour.
   const uint64_t dQ = smem_desc(smem_u32(sQ), 16, 8 * C::ROWB, C::LAYOUT);
   const uint64_t dK = smem_desc(smem_u32(sKV), 16, 8 * C::ROWB, C::LAYOUT);
   const uint64_t dV = F8 ? smem_desc(smem_u32(sKV), 16, 8 * C::ROWB, C::LAYOUT)
-                        : smem_desc(smem_u32(sKV), C::KV_CHUNK_BYTES, 8 * C::ROWB, C::LAYOUT);
+                        : smem_desc(smem_u32(sKV), C::V_CHUNK_BYTES, 8 * C::ROWB, C::LAYOUT);
   // S[slot] = Q_qt K^T : A = Q tile (K-major), B = K tile (K-major), k-steps of 16 along d.
   auto issue_qk = [&](int qt, int s_col, int stage) {
     const uint64_t a0 = dQ + uint64_t((qt * C::Q_TILE_BYTES) >> 4);
@@ -278,23 +298,13 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
 #pragma unroll
     for (int kk = 0; kk < D / C::KSTEP; ++kk) {
       const uint32_t ao = (kk / C::KPC) * C::Q_CHUNK_BYTES + (kk % C::KPC) * 32;
-      const uint32_t bo = (kk / C::KPC) * C::KV_CHUNK_BYTES + (kk % C::KPC) * 32;
-      if (F8)
+      const uint32_t bo = (kk / C::KPC) * C::K_CHUNK_BYTES + (kk % C::KPC) * 32;
+      if (PAIR)
+        umma_ss_pair(tmem + s_col, a0 + (ao >> 4), b0 + (bo >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+      else if (F8)
         umma_ss_f8(tmem + s_col, a0 + (ao >> 4), b0 + (bo >> 4), idesc_qk, kk > 0 ? 1u : 0u);
-      else if (C::Q_TMEM)
-        umma_ts(tmem + s_col, tmem + C::Q_COL + kk * 8, b0 + (bo >> 4), idesc_qk, kk > 0 ? 1u : 0u);
       else
         umma_ss(tmem + s_col, a0 + (ao >> 4), b0 + (bo >> 4), idesc_qk, kk > 0 ? 1u : 0u);
-    }
-  };
-  // Q tile -> TMEM (one 128-row x 16-element block per k-step, from the same shared-memory
-  // descriptor the QK would read it through). tcgen05.cp and tcgen05.mma issued by one thread run
-  // in issue order, so the copy lands after the previous unit's last QK and before this unit's.
-  auto copy_q_to_tmem = [&]() {
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t ao = (kk / C::KPC) * C::Q_CHUNK_BYTES + (kk % C::KPC) * 32;
-      tmem_cp_128x256b(tmem + C::Q_COL + kk * 8, dQ + (ao >> 4));
     }
   };
   // O += P V over the tile's keys: A = P (bf16, in TMEM over S), B = V tile read MN-major (N = d),
@@ -305,7 +315,10 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
     for (int kk = 0; kk < C::BN / C::KSTEP; ++kk) {
       // A = P: KSTEP keys = 8 TMEM columns in both forms; B: the next KSTEP rows of V (MN-major) or
       // the next 32 bytes of each transposed-V row (K-major)
-      if (F8)
+      if (PAIR)
+        umma_ts_pair(tmem + o_col, tmem + p_col + kk * 8, b0 + uint64_t((kk * 16 * C::ROWB) >> 4), idesc_pv,
+                     (accumulate || kk > 0) ? 1u : 0u);
+      else if (F8)
         umma_ts_f8(tmem + o_col, tmem + p_col + kk * 8, b0 + uint64_t((kk * 32) >> 4), idesc_pv,
                    (accumulate || kk > 0) ? 1u : 0u);
       else
@@ -331,6 +344,23 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
     if (!whole_warp || lane == 0) mbar_arrive(&sched_empty[slot]);
     return lin;
   };
+  // A pair's units are fixed instead: cluster p of P takes units p, p + P, p + 2P, ... in issue
+  // order, and every role of both CTAs walks the same list.
+  auto pair_unit = [&](int k) -> int {
+    const long long lin = (long long)(blockIdx.x / 2) + (long long)k * (gridDim.x / 2);
+    return lin < total_units ? int(lin) : -1;
+  };
+  // MMA completion: to this CTA's barrier, or to the barrier at the same offset in both CTAs of a pair
+  auto commit = [&](uint64_t* bar) {
+    if (PAIR)
+      umma_commit_pair(bar);
+    else
+      umma_commit(bar);
+  };
+  // waits on phases that the other CTA of a pair may complete (acquire at cluster scope)
+  auto wait_x = [&](uint64_t* bar, uint32_t ph) -> bool {
+    return PAIR ? mbar_wait_cluster(bar, ph, abort_flag, T) : mbar_wait(bar, ph, abort_flag, T);
+  };
 
   if (warp == 0) {
     // ================================ TMA producer ================================
@@ -340,40 +370,74 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
       int pos = 0;  // next ring position
       int qc = 0;   // units loaded so far (phase of q_full / q_empty)
       for (int k = 0; ok; ++k) {
-        // claim the next unit (longest first) and hand it to the other roles
-        const int slot = k % C::SCHED;
-        if (!mbar_wait(&sched_empty[slot], uint32_t(((k / C::SCHED) & 1) ^ 1), abort_flag, T)) {
-          ok = false;
-          break;
+        int lin;
+        if (PAIR) {
+          lin = pair_unit(k);
+        } else {
+          // claim the next unit (longest first) and hand it to the other roles
+          const int slot = k % C::SCHED;
+          if (!mbar_wait(&sched_empty[slot], uint32_t(((k / C::SCHED) & 1) ^ 1), abort_flag, T)) {
+            ok = false;
+            break;
+          }
+          const unsigned claimed = atomicAdd(&g_sched_next[args.sched_slot], 1u);
+          lin = claimed < unsigned(total_units) ? int(claimed) : -1;
+          sched_unit[slot] = lin;
+          mbar_arrive(&sched_full[slot]);
         }
-        const unsigned claimed = atomicAdd(&g_sched_next[args.sched_slot], 1u);
-        const int lin = claimed < unsigned(total_units) ? int(claimed) : -1;
-        sched_unit[slot] = lin;
-        mbar_arrive(&sched_full[slot]);
         if (lin < 0) break;
-        const Unit un = unit_at<D>(args, lin);
+        const Unit un = unit_at<D, PAIR>(args, lin);
         if (un.n_tiles == 0) continue;
         const int g = un.h / args.group;
         // Q of the previous unit must be consumed by all its QK MMAs before it is overwritten
-        if (qc > 0 && !mbar_wait(q_empty, (qc - 1) & 1, abort_flag, T)) {
+        if (qc > 0 && !wait_x(q_empty, (qc - 1) & 1)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(q_full, C::NQT * C::Q_TILE_BYTES);
-#pragma unroll
-        for (int qt = 0; qt < C::NQT; ++qt)
+        if (PAIR) {
+          // each CTA loads its own 128 rows; the leader's q_full counts the bytes of both
+          if (rank == 0) mbar_arrive_expect_tx_local(q_full, C::CTAS * C::Q_TILE_BYTES);
+          const uint32_t bar_l = mapa_shared(q_full, 0);
 #pragma unroll
           for (int c = 0; c < C::NCHUNK; ++c)
-            tma_load_4d(sQ + qt * C::Q_TILE_BYTES + c * C::Q_CHUNK_BYTES, &tmQ, q_full, c * C::CHUNK, un.h,
-                        un.q0 + qt * C::BM, un.b);
+            tma_load_4d_pair(sQ + c * C::Q_CHUNK_BYTES, &tmQ, bar_l, c * C::CHUNK, un.h, un.q0 + int(rank) * C::BM,
+                             un.b);
+        } else {
+          mbar_arrive_expect_tx(q_full, C::NQT * C::Q_TILE_BYTES);
+#pragma unroll
+          for (int qt = 0; qt < C::NQT; ++qt)
+#pragma unroll
+            for (int c = 0; c < C::NCHUNK; ++c)
+              tma_load_4d(sQ + qt * C::Q_TILE_BYTES + c * C::Q_CHUNK_BYTES, &tmQ, q_full, c * C::CHUNK, un.h,
+                          un.q0 + qt * C::BM, un.b);
+        }
         ++qc;
         for (int j = 0; j < un.n_tiles && ok; ++j) {
 #pragma unroll
           for (int kv = 0; kv < 2; ++kv, ++pos) {
             const int s = kv_slot(pos);
-            if (!mbar_wait(&kv_empty[s], kv_phase(pos) ^ 1, abort_flag, T)) {
+            if (!wait_x(&kv_empty[s], kv_phase(pos) ^ 1)) {
               ok = false;
               break;
+            }
+            if (PAIR) {
+              // K part: this CTA's 64 keys of the tile, all of d; V part: all keys, this CTA's half of d.
+              // The leader's kv_full counts the bytes of both CTAs.
+              if (rank == 0) mbar_arrive_expect_tx_local(&kv_full[s], C::CTAS * C::KV_TILE_BYTES);
+              const uint32_t bar_l = mapa_shared(&kv_full[s], 0);
+              uint8_t* dst = sKV + s * C::KV_TILE_BYTES;
+              if (kv == 0) {
+#pragma unroll
+                for (int c = 0; c < C::NCHUNK; ++c)
+                  tma_load_4d_pair(dst + c * C::K_CHUNK_BYTES, &tmK, bar_l, c * C::CHUNK, g,
+                                   j * C::BN + int(rank) * C::K_ROWS, un.b);
+              } else {
+#pragma unroll
+                for (int c = 0; c < C::V_COLS / C::CHUNK; ++c)
+                  tma_load_4d_pair(dst + c * C::V_CHUNK_BYTES, &tmV, bar_l, int(rank) * C::V_COLS + c * C::CHUNK, g,
+                                   j * C::BN, un.b);
+              }
+              continue;
             }
             mbar_arrive_expect_tx(&kv_full[s], C::KV_TILE_BYTES);
             const CUtensorMap* m = kv ? &tmV : &tmK;
@@ -383,14 +447,15 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
             } else {
 #pragma unroll
               for (int c = 0; c < C::NCHUNK; ++c)
-                tma_load_4d(sKV + s * C::KV_TILE_BYTES + c * C::KV_CHUNK_BYTES, m, &kv_full[s], c * C::CHUNK, g,
+                tma_load_4d(sKV + s * C::KV_TILE_BYTES + c * C::K_CHUNK_BYTES, m, &kv_full[s], c * C::CHUNK, g,
                             j * C::BN, un.b);
             }
           }
         }
       }
-      if (!ok) {
-        // Give the copies already in flight a bounded chance to land before the CTA exits.
+      if (!ok && rank == 0) {
+        // Give the copies already in flight a bounded chance to land before the CTA exits (a pair's
+        // copies, the peer's included, complete on the leader's barriers).
         if (qc > 0) mbar_wait(q_full, (qc - 1) & 1, nullptr, 100000000ull);
         // ring positions [0, pos) were issued; slot s holds the fills at positions s, s + STAGES, ...
         for (int s = 0; s < C::STAGES; ++s) {
@@ -403,7 +468,7 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
   } else if (warp == 1) {
     // ================================ MMA issuer ================================
     if (kSplitRegs) regs_dec<C::CTRL_REGS>();
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {  // a pair: the leader issues for both CTAs
       // K/V tiles and Q arrive by TMA (complete_tx on the mbarrier): the MMAs may read them once the
       // barrier phase is observed. P is written to TMEM by the softmax threads' tcgen05.st, so
       // observing p_full is followed by tcgen05.fence::after_thread_sync before the PV MMAs.
@@ -414,17 +479,13 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
       int qk_cnt[2] = {0, 0};  // separate P: S tiles issued per query tile (phase of s_free)
       int t_run = 0;  // single-tile path: S tiles issued so far (slot = t_run & 1)
       for (int k = 0; ok; ++k) {
-        const int lin = next_unit(k, false);
+        const int lin = PAIR ? pair_unit(k) : next_unit(k, false);
         if (lin < 0) break;
-        const Unit un = unit_at<D>(args, lin);
+        const Unit un = unit_at<D, PAIR>(args, lin);
         const int n = un.n_tiles;
         if (n == 0) continue;
-        ok = mbar_wait(q_full, qc & 1, abort_flag, T);
+        ok = wait_x(q_full, qc & 1);
         ++qc;
-        if (C::Q_TMEM && ok) {
-          copy_q_to_tmem();
-          umma_commit(q_empty);  // shared-memory Q is free once the copy is done
-        }
         const int base = pos;  // K_j at base + 2j, V_j at base + 2j + 1
         if (C::SEP_P) {
           // Two query tiles, P in buffers of its own. QK(t, j+1) may overwrite S once the softmax has
@@ -433,47 +494,47 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
           const int nt[2] = {un.n_tile0, n};
           auto qk_into = [&](int qt, int jj, int stage) -> bool {
             if (qk_cnt[qt] > 0) {
-              if (!mbar_wait(&s_free[qt], uint32_t((qk_cnt[qt] - 1) & 1), abort_flag, T)) return false;
+              if (!wait_x(&s_free[qt], uint32_t((qk_cnt[qt] - 1) & 1))) return false;
               tc_fence_after();
             }
             issue_qk(qt, qt ? C::S_COL1 : C::S_COL0, stage);
-            umma_commit(&s_full[qt]);
-            if (qt == 1 && jj == n - 1) umma_commit(q_empty);  // the unit's last QK: Q may be reloaded
+            commit(&s_full[qt]);
+            if (qt == 1 && jj == n - 1) commit(q_empty);  // the unit's last QK: Q may be reloaded
             ++qk_cnt[qt];
             return true;
           };
-          if (ok) ok = mbar_wait(&kv_full[kv_slot(base)], kv_phase(base), abort_flag, T);
+          if (ok) ok = wait_x(&kv_full[kv_slot(base)], kv_phase(base));
 #pragma unroll
           for (int qt = 0; qt < 2; ++qt)
             if (ok && nt[qt] > 0) ok = qk_into(qt, 0, kv_slot(base));
-          if (ok) umma_commit(&kv_empty[kv_slot(base)]);
+          if (ok) commit(&kv_empty[kv_slot(base)]);
           for (int j = 0; j < n && ok; ++j) {
             const int pv_pos = base + 2 * j + 1, pk_pos = base + 2 * j + 2;
             const bool nxt = j + 1 < n;
-            ok = mbar_wait(&kv_full[kv_slot(pv_pos)], kv_phase(pv_pos), abort_flag, T);
-            if (ok && nxt) ok = mbar_wait(&kv_full[kv_slot(pk_pos)], kv_phase(pk_pos), abort_flag, T);
+            ok = wait_x(&kv_full[kv_slot(pv_pos)], kv_phase(pv_pos));
+            if (ok && nxt) ok = wait_x(&kv_full[kv_slot(pk_pos)], kv_phase(pk_pos));
 #pragma unroll
             for (int qt = 0; qt < 2; ++qt)
               if (ok && j + 1 < nt[qt]) ok = qk_into(qt, j + 1, kv_slot(pk_pos));
 #pragma unroll
             for (int qt = 0; qt < 2; ++qt) {
               if (!ok || j >= nt[qt]) continue;
-              ok = mbar_wait(&p_full[qt], pc[qt] & 1, abort_flag, T);
+              ok = wait_x(&p_full[qt], pc[qt] & 1);
               if (!ok) break;
               ++pc[qt];
               tc_fence_after();
               issue_pv(qt ? C::O_COL1 : C::O_COL0, qt ? C::P_COL1 : C::P_COL0, kv_slot(pv_pos), j > 0);
-              umma_commit(&p_free[qt]);
-              if (qt == 0 && j == nt[0] - 1 && nt[0] < n) umma_commit(&o_final[0]);  // see below
+              commit(&p_free[qt]);
+              if (qt == 0 && j == nt[0] - 1 && nt[0] < n) commit(&o_final[0]);  // see below
             }
             if (!ok) break;
-            umma_commit(&kv_empty[kv_slot(pv_pos)]);
-            if (nxt) umma_commit(&kv_empty[kv_slot(pk_pos)]);
+            commit(&kv_empty[kv_slot(pv_pos)]);
+            if (nxt) commit(&kv_empty[kv_slot(pk_pos)]);
           }
           pos = base + 2 * n;
         } else if (C::NQT == 2) {
           // Two query tiles, one S slot each: QK(0,0) QK(1,0) | PV(0,j) QK(0,j+1) PV(1,j) QK(1,j+1) | ...
-          if (ok) ok = mbar_wait(&kv_full[kv_slot(base)], kv_phase(base), abort_flag, T);
+          if (ok) ok = wait_x(&kv_full[kv_slot(base)], kv_phase(base));
           // a causal unit's first query tile may need one K/V tile fewer than the second
           const int nt[2] = {un.n_tile0, n};
           if (ok) {
@@ -481,70 +542,70 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
             for (int qt = 0; qt < 2; ++qt) {
               if (nt[qt] == 0) continue;
               issue_qk(qt, qt ? C::S_COL1 : C::S_COL0, kv_slot(base));
-              umma_commit(&s_full[qt]);
-              if (qt == 1 && n == 1) umma_commit(q_empty);  // the unit's last QK: Q may be reloaded
+              commit(&s_full[qt]);
+              if (qt == 1 && n == 1) commit(q_empty);  // the unit's last QK: Q may be reloaded
             }
-            umma_commit(&kv_empty[kv_slot(base)]);
+            commit(&kv_empty[kv_slot(base)]);
           }
           for (int j = 0; j < n && ok; ++j) {
             const int pv_pos = base + 2 * j + 1, pk_pos = base + 2 * j + 2;
             const bool nxt = j + 1 < n;
-            ok = mbar_wait(&kv_full[kv_slot(pv_pos)], kv_phase(pv_pos), abort_flag, T);
-            if (ok && nxt) ok = mbar_wait(&kv_full[kv_slot(pk_pos)], kv_phase(pk_pos), abort_flag, T);
+            ok = wait_x(&kv_full[kv_slot(pv_pos)], kv_phase(pv_pos));
+            if (ok && nxt) ok = wait_x(&kv_full[kv_slot(pk_pos)], kv_phase(pk_pos));
 #pragma unroll
             for (int qt = 0; qt < 2; ++qt) {
               if (!ok) break;
               if (j >= nt[qt]) continue;
               const int s_col = qt ? C::S_COL1 : C::S_COL0;
-              ok = mbar_wait(&p_full[qt], pc[qt] & 1, abort_flag, T);
+              ok = wait_x(&p_full[qt], pc[qt] & 1);
               if (!ok) break;
               ++pc[qt];
               tc_fence_after();
               issue_pv(qt ? C::O_COL1 : C::O_COL0, s_col, kv_slot(pv_pos), j > 0);
-              if (qt == 0 && j == nt[0] - 1 && nt[0] < n) umma_commit(&o_final[0]);  // see below
+              if (qt == 0 && j == nt[0] - 1 && nt[0] < n) commit(&o_final[0]);  // see below
               // P of this tile is consumed by the PV MMAs above before this QK overwrites the slot:
               // MMAs issued by one thread execute in issue order.
               if (j + 1 < nt[qt]) {
                 issue_qk(qt, s_col, kv_slot(pk_pos));
-                umma_commit(&s_full[qt]);
-                if (qt == 1 && j + 2 == n) umma_commit(q_empty);  // the unit's last QK
+                commit(&s_full[qt]);
+                if (qt == 1 && j + 2 == n) commit(q_empty);  // the unit's last QK
               }
             }
             if (!ok) break;
-            umma_commit(&kv_empty[kv_slot(pv_pos)]);
-            if (nxt) umma_commit(&kv_empty[kv_slot(pk_pos)]);
+            commit(&kv_empty[kv_slot(pv_pos)]);
+            if (nxt) commit(&kv_empty[kv_slot(pk_pos)]);
           }
           pos = base + 2 * n;
         } else {
           // One query tile, S alternating between two slots: QK_0, QK_1, PV_0, QK_2, PV_1, QK_3, ...
           const int t0 = t_run;
           for (int j = 0; j < 2 && j < n && ok; ++j) {
-            ok = mbar_wait(&kv_full[kv_slot(base + 2 * j)], kv_phase(base + 2 * j), abort_flag, T);
+            ok = wait_x(&kv_full[kv_slot(base + 2 * j)], kv_phase(base + 2 * j));
             if (!ok) break;
             issue_qk(0, ((t0 + j) & 1) ? C::S_COL1 : C::S_COL0, kv_slot(base + 2 * j));
-            umma_commit(&s_full[(t0 + j) & 1]);
-            if (!C::Q_TMEM && j == n - 1) umma_commit(q_empty);  // the unit's last QK: Q may be reloaded
-            umma_commit(&kv_empty[kv_slot(base + 2 * j)]);
+            commit(&s_full[(t0 + j) & 1]);
+            if (j == n - 1) commit(q_empty);  // the unit's last QK: Q may be reloaded
+            commit(&kv_empty[kv_slot(base + 2 * j)]);
           }
           for (int j = 0; j < n && ok; ++j) {
             const int t = t0 + j;
             const int slot = t & 1;
             const int s_col = slot ? C::S_COL1 : C::S_COL0;
-            ok = mbar_wait(&kv_full[kv_slot(base + 2 * j + 1)], kv_phase(base + 2 * j + 1), abort_flag, T);
-            if (ok) ok = mbar_wait(&p_full[slot], (t >> 1) & 1, abort_flag, T);
+            ok = wait_x(&kv_full[kv_slot(base + 2 * j + 1)], kv_phase(base + 2 * j + 1));
+            if (ok) ok = wait_x(&p_full[slot], (t >> 1) & 1);
             if (!ok) break;
             tc_fence_after();
             issue_pv(C::O_COL0, s_col, kv_slot(base + 2 * j + 1), j > 0);
-            umma_commit(o_done);
-            umma_commit(&kv_empty[kv_slot(base + 2 * j + 1)]);
+            commit(o_done);
+            commit(&kv_empty[kv_slot(base + 2 * j + 1)]);
             if (j + 2 < n) {
               const int kp = base + 2 * (j + 2);
-              ok = mbar_wait(&kv_full[kv_slot(kp)], kv_phase(kp), abort_flag, T);
+              ok = wait_x(&kv_full[kv_slot(kp)], kv_phase(kp));
               if (!ok) break;
               issue_qk(0, s_col, kv_slot(kp));
-              umma_commit(&s_full[slot]);
-              if (!C::Q_TMEM && j + 3 == n) umma_commit(q_empty);  // the unit's last QK
-              umma_commit(&kv_empty[kv_slot(kp)]);
+              commit(&s_full[slot]);
+              if (j + 3 == n) commit(q_empty);  // the unit's last QK
+              commit(&kv_empty[kv_slot(kp)]);
             }
           }
           t_run = t0 + n;
@@ -556,12 +617,12 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
         // after its own last PV instead, so its epilogue runs during tile 1's last step. (Q was
         // released after the unit's last QK, so the next unit's Q load overlaps the last PVs and the
         // epilogues.)
-        if (C::NQT == 1 || un.n_tile0 == 0 || un.n_tile0 == n) umma_commit(&o_final[0]);
-        if (C::NQT == 2) umma_commit(&o_final[1]);
+        if (C::NQT == 1 || un.n_tile0 == 0 || un.n_tile0 == n) commit(&o_final[0]);
+        if (C::NQT == 2) commit(&o_final[1]);
       }
       if (!ok) {
         // Let the MMAs already issued finish before tensor memory is released.
-        umma_commit(drain);
+        commit(drain);
         mbar_wait(drain, 0, nullptr, 100000000ull);
       }
     }
@@ -582,8 +643,17 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
     float o_mul = 1.0f;         // epilogue factor on O (8-bit: V's dequantization)
     // every lane waits; the warp continues only if all of them saw the phase (tcgen05.ld/st below are
     // warp-collective, so a partial give-up must not split the warp)
-    auto wait_warp = [&](uint64_t* bar, uint32_t ph) -> bool {
-      return __all_sync(0xffffffffu, mbar_wait(bar, ph, abort_flag, T));
+    auto wait_warp = [&](uint64_t* bar, uint32_t ph) -> bool { return __all_sync(0xffffffffu, wait_x(bar, ph)); };
+    // P of this warp's 32 rows is in TMEM: tell the MMA thread (a pair's is in the leader)
+    auto publish_p = [&](uint64_t* bar) {
+      if (PAIR) {
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(bar, 0));
+      } else {
+        warp_publish_tmem_stores(bar, lane);
+      }
     };
 
     bool ok = true;
@@ -592,9 +662,9 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
     int uc = 0;     // units with keys finished (phase of o_final)
     int pt = 0;     // separate P: P tiles this warpgroup has published (phase of p_free[qt])
     for (int k = 0; ok; ++k) {
-      const int lin = next_unit(k, true);
+      const int lin = PAIR ? pair_unit(k) : next_unit(k, true);
       if (lin < 0) break;
-      const Unit un = unit_at<D>(args, lin);
+      const Unit un = unit_at<D, PAIR>(args, lin);
       if (F8) {
         // codes decode as value = code * amax / 448 per (batch, head)
         const int g = un.h / args.group;
@@ -604,7 +674,7 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
         sc_nat = args.scale * dq * dk;
         o_mul = args.amax_v[un.b * args.Hkv + g] / 448.0f;
       }
-      const int q_first = un.q0 + qt * C::BM;
+      const int q_first = un.q0 + (qt + int(rank)) * C::BM;  // (a pair: NQT = 1, rank 1 takes the second 128 rows)
       const int q_row = q_first + row;
       // last key visible to this row (any key index <= lim is visible); rows past Nq are padding
       const int lim = args.causal ? min(args.Nkv - 1, q_row + diag) : args.Nkv - 1;
@@ -773,7 +843,7 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
           else
             tmem_st16(p_addr + half * C::HALF_PAIRS, p);
         }
-        warp_publish_tmem_stores(&p_full[slot], lane);
+        publish_p(&p_full[slot]);
         ++pt;
         const float2 s01 = fadd2(acc4[0], acc4[1]);
         const float2 s23 = fadd2(acc4[2], acc4[3]);
@@ -836,12 +906,18 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  // a pair: neither CTA frees its tensor memory or exits while the leader's MMAs or the other CTA's
+  // barrier arrivals and copies may still reach it
+  if (PAIR) cluster_sync();
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    if (PAIR)
+      tmem_dealloc_pair(tmem, C::TMEM_COLS);
+    else
+      tmem_dealloc(tmem, C::TMEM_COLS);
   }
   // The last CTA to finish returns the scheduling slot to zero (all CTAs have stopped claiming).
-  if (threadIdx.x == 0) {
+  if (!PAIR && threadIdx.x == 0) {
     __threadfence();
     if (atomicAdd(&g_sched_done[args.sched_slot], 1u) == gridDim.x - 1) {
       atomicExch(&g_sched_next[args.sched_slot], 0u);
@@ -855,11 +931,12 @@ __global__ void __launch_bounds__(FwdCfg<D, F8>::THREADS, 1)
 // ---------------------------------------------------------------------------------------------
 // F8: q and k are e4m3 codes [B, N, H, d], v is the transposed code tensor [B, Hkv, d, Nkv] and
 // amax_* the per-(batch, head) dequantization maxima; otherwise bf16 tensors and null amax.
-template <int D, bool F8>
+template <int D, bool F8, bool PAIR = false>
 static attn_status_t launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                                 int Hkv, int Nq, int Nkv, float scale, int causal, const float* amax_q,
                                 const float* amax_k, const float* amax_v, cudaStream_t stream) {
-  using C = FwdCfg<D, F8>;
+  using C = FwdCfg<D, F8, PAIR>;
+  auto kernel = attn_fwd_kernel<D, F8, PAIR>;
   CUtensorMap tmQ, tmK, tmV;
   const uint32_t swz = C::ROWB == 128 ? 128u : 64u;
   if (F8) {
@@ -869,12 +946,12 @@ static attn_status_t launch_fwd(const void* q, const void* k, const void* v, voi
         !encode_map(&tmV, v, 1, dvt, bv, swz))
       return ATTN_ERR_CUDA;
   } else if (!encode_tile_map(&tmQ, q, D, Hq, Nq, B, C::CHUNK, C::BM, swz) ||
-             !encode_tile_map(&tmK, k, D, Hkv, Nkv, B, C::CHUNK, C::BN, swz) ||
+             !encode_tile_map(&tmK, k, D, Hkv, Nkv, B, C::CHUNK, C::K_ROWS, swz) ||
              !encode_tile_map(&tmV, v, D, Hkv, Nkv, B, C::CHUNK, C::BN, swz)) {
     return ATTN_ERR_CUDA;
   }
 
-  if (ensure_dyn_smem(reinterpret_cast<const void*>(attn_fwd_kernel<D, F8>), C::SMEM_BYTES) != cudaSuccess)
+  if (ensure_dyn_smem(reinterpret_cast<const void*>(kernel), C::SMEM_BYTES) != cudaSuccess)
     return ATTN_ERR_CUDA;
   // setmaxnreg.inc waits until the registers it asks for are free in the CTA's launch allocation,
   // so a split whose total exceeds that allocation would never proceed: refuse to launch it.
@@ -883,7 +960,7 @@ static attn_status_t launch_fwd(const void* q, const void* k, const void* v, voi
     int st = regs_ok.load(std::memory_order_relaxed);
     if (st == 0) {
       cudaFuncAttributes fa;
-      if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, F8>) != cudaSuccess) return ATTN_ERR_CUDA;
+      if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return ATTN_ERR_CUDA;
       const long long pool = (long long)fa.numRegs * C::THREADS;
       const long long need = 128LL * C::CTRL_REGS + 128LL * C::NSMWG * C::SM_REGS;
       st = pool >= need ? 1 : 2;
@@ -900,7 +977,7 @@ static attn_status_t launch_fwd(const void* q, const void* k, const void* v, voi
   a.Nq = Nq;
   a.Nkv = Nkv;
   a.group = Hq / Hkv;
-  a.n_qblk = (Nq + C::NQT * C::BM - 1) / (C::NQT * C::BM);
+  a.n_qblk = (Nq + C::UNIT_ROWS - 1) / C::UNIT_ROWS;
   a.causal = causal;
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
@@ -923,13 +1000,38 @@ static attn_status_t launch_fwd(const void* q, const void* k, const void* v, voi
   }
   const long long units = (long long)a.n_qblk * B * Hq;
   if (units > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
-  // persistent grid: one CTA per SM (each holds all 512 TMEM columns), walking the units in order
   const int sms = sm_count();
   if (sms <= 0) return ATTN_ERR_CUDA;
+  if (PAIR) {
+    // persistent grid of CTA pairs: as many pairs as fit on the device at once (one CTA per SM), each
+    // walking its fixed share of the units
+    const int pairs = max_pairs(reinterpret_cast<const void*>(kernel), C::THREADS, C::SMEM_BYTES);
+    if (pairs <= 0) return ATTN_ERR_CUDA;
+    const long long n_pairs = units < pairs ? units : pairs;
+    a.sched_slot = 0;
+    cudaLaunchConfig_t lc = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    lc.gridDim = dim3(unsigned(2 * n_pairs));
+    lc.blockDim = dim3(C::THREADS);
+    lc.dynamicSmemBytes = C::SMEM_BYTES;
+    lc.stream = stream;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&lc, kernel, tmQ, tmK, tmV, a) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+  }
+  // persistent grid: one CTA per SM (each holds all 512 TMEM columns), walking the units in order
   const unsigned grid = unsigned(units < sms ? units : sms);
   static std::atomic<unsigned> launch_count{0};
   a.sched_slot = int(launch_count.fetch_add(1) % kSchedSlots);
-  attn_fwd_kernel<D, F8><<<dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, a);
+  kernel<<<dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, a);
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
 }
 
@@ -939,7 +1041,7 @@ attn_status_t fwd_dispatch(const void* q, const void* k, const void* v, void* o,
     case 32: return launch_fwd<32, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, nullptr, nullptr, nullptr, stream);
     case 64: return launch_fwd<64, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, nullptr, nullptr, nullptr, stream);
     case 128: return launch_fwd<128, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, nullptr, nullptr, nullptr, stream);
-    case 256: return launch_fwd<256, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, nullptr, nullptr, nullptr, stream);
+    case 256: return launch_fwd<256, false, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, nullptr, nullptr, nullptr, stream);
     default: return ATTN_ERR_UNSUPPORTED;
   }
 }

@@ -43,6 +43,9 @@ constexpr int kMaxDevices = 128;
 
 // Streaming multiprocessors of the current device (-1 on error), looked up once per device.
 int sm_count();
+// Clusters of two CTAs of `func` (threads, dynamic shared memory as given) resident on the current
+// device at once; cached per device for the last kernel asked about. -1 on error.
+int max_pairs(const void* func, int threads, int smem_bytes);
 
 // A 4-d TMA map over a token-major bf16 tensor [outer, rows, heads, d] (d innermost), with a box
 // of `box_cols` elements of d x 1 head x `box_rows` tokens x 1 batch; swizzle_bytes is 128, 64 or 0

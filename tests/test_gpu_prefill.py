@@ -66,6 +66,19 @@ def test_large_score_spread(lib):
     _run_small(lib, 4102, 1, 2, 2, 384, 384, 256, True, scale=1.5)
 
 
+def test_head_dim_256_cta_pairs(lib):
+    # d = 256 runs on CTA pairs: 256 query rows per unit, 128 in each CTA, 128-key tiles split between
+    # the two. 100 rows leave the second CTA without a valid row and 130 with two; 300 keys end in a
+    # ragged tile whose two halves are partly and wholly past the end; 2 x 8 x 6 = 96 causal units on
+    # at most 74 pairs give pairs several units, so the hand-off counters carry across units (twice
+    # 1/sqrt(d) makes the running max move often; much larger scales make P nearly one-hot and O a
+    # single V row, whose bf16 rounding alone can exceed the gate at every head dim).
+    _run_small(lib, 4500, 1, 2, 1, 100, 300, 256, False)
+    _run_small(lib, 4501, 1, 2, 2, 130, 130, 256, True)
+    _run_small(lib, 4502, 1, 2, 2, 1, 193, 256, False)
+    _run_small(lib, 4503, 2, 8, 4, 1300, 1300, 256, True, scale=0.125)
+
+
 @pytest.mark.parametrize("d", [32, 64])
 def test_small_head_dims_rescale_and_units_per_cta(lib, d):
     # d <= 64 keeps P in buffers of its own; a large scale makes the running max jump (O rescales that
