@@ -69,18 +69,21 @@ constexpr float kRescaleTau = 8.0f;
 
 // F8: Q and K are e4m3 codes (rotated), V is given transposed (e4m3 [d, keys] per head), and the
 // products run as kind::f8f6f4 MMAs with 32-element k-steps; P is packed four e4m3 per TMEM column.
-// PAIR (d = 256): a cluster of two CTAs works on 256 query rows, 128 per CTA, with 2-SM MMAs
+// PAIR (used at d = 256): a cluster of two CTAs works on 256 query rows, 128 per CTA, with 2-SM MMAs
 // (cta_group::2, M = 256). Each CTA holds half of every K tile (its 64 of the tile's 128 keys) and
 // half of every V tile (its 128 of the d columns), so 128-key tiles fit a 5-stage ring and the QK
 // products run at N = 128 (a 64-key N = 64 product costs ~52 cycles per k-step against 32 for its
-// FLOPs; N = 128 runs at the full rate).
+// FLOPs; N = 128 runs at the full rate). The same configuration builds at d = 128 (one query tile per
+// CTA, two S slots) but measured slower there than two query tiles per CTA: with half the FLOPs per
+// key tile, the single softmax warpgroup per CTA sets the pace.
 template <int D, bool F8 = false, bool PAIR = false>
 struct FwdCfg {
   static_assert(!F8 || D == 128, "the 8-bit path is built for d = 128");
-  static_assert(PAIR == (D == 256), "d = 256 runs on CTA pairs, d <= 128 on single CTAs");
+  static_assert(!PAIR || (D >= 128 && !F8), "CTA pairs are built for bf16 at d = 128 and 256");
+  static_assert(PAIR || D <= 128, "d = 256 runs on CTA pairs");
   static constexpr int EB = F8 ? 1 : 2;                 // bytes per element of Q, K, V
   static constexpr int BM = 128;                        // query rows per tile (TMEM lanes)
-  static constexpr int NQT = (D <= 128) ? 2 : 1;        // query tiles per CTA
+  static constexpr int NQT = (D <= 128 && !PAIR) ? 2 : 1;  // query tiles per CTA
   static constexpr int BN = (D <= 128 || PAIR) ? 128 : 64;  // keys per K/V tile
   static constexpr int CTAS = PAIR ? 2 : 1;             // CTAs per unit
   static constexpr int UNIT_ROWS = NQT * BM * CTAS;     // query rows per unit
@@ -395,8 +398,10 @@ __global__ void __launch_bounds__(FwdCfg<D, F8, PAIR>::THREADS, 1)
           break;
         }
         if (PAIR) {
-          // each CTA loads its own 128 rows; the leader's q_full counts the bytes of both
-          if (rank == 0) mbar_arrive_expect_tx_local(q_full, C::CTAS * C::Q_TILE_BYTES);
+          // each CTA loads its own 128 rows; the leader's q_full counts the bytes of both (the leader
+          // arrives on its own barrier, so the plain CTA-scope form suffices: a cluster-scope release
+          // costs ~1,000 cycles on this path)
+          if (rank == 0) mbar_arrive_expect_tx(q_full, C::CTAS * C::Q_TILE_BYTES);
           const uint32_t bar_l = mapa_shared(q_full, 0);
 #pragma unroll
           for (int c = 0; c < C::NCHUNK; ++c)
@@ -423,7 +428,7 @@ __global__ void __launch_bounds__(FwdCfg<D, F8, PAIR>::THREADS, 1)
             if (PAIR) {
               // K part: this CTA's 64 keys of the tile, all of d; V part: all keys, this CTA's half of d.
               // The leader's kv_full counts the bytes of both CTAs.
-              if (rank == 0) mbar_arrive_expect_tx_local(&kv_full[s], C::CTAS * C::KV_TILE_BYTES);
+              if (rank == 0) mbar_arrive_expect_tx(&kv_full[s], C::CTAS * C::KV_TILE_BYTES);
               const uint32_t bar_l = mapa_shared(&kv_full[s], 0);
               uint8_t* dst = sKV + s * C::KV_TILE_BYTES;
               if (kv == 0) {
@@ -1040,7 +1045,7 @@ attn_status_t fwd_dispatch(const void* q, const void* k, const void* v, void* o,
   switch (d) {
     case 32: return launch_fwd<32, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, nullptr, nullptr, nullptr, stream);
     case 64: return launch_fwd<64, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, nullptr, nullptr, nullptr, stream);
-    case 128: return launch_fwd<128, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, nullptr, nullptr, nullptr, stream);
+    case 128: return launch_fwd<128, false, false>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, nullptr, nullptr, nullptr, stream);
     case 256: return launch_fwd<256, false, true>(q, k, v, o, lse, B, Hq, Hkv, Nq, Nkv, scale, causal, nullptr, nullptr, nullptr, stream);
     default: return ATTN_ERR_UNSUPPORTED;
   }
