@@ -46,26 +46,32 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 # that file changes, the figure is stale and the bench line reports null until it is measured again.
 PREFILL_SRC = "exact_io_aware_41_b200/csrc/attn_fwd.cu"
 DECODE_SRC = "exact_io_aware_41_b200/csrc/attn_decode.cu"
-PREFILL_SHA = "ab469009540e1a218be3af0398ce49023e016c49ac7226da759dd84960e98ae8"  # sha256 of PREFILL_SRC when the prefill figures were taken
+PREFILL_SHA = "0f72f8309b2d52a6219e56f70d6a4c9da93d023415cbe62689bc13f787aae103"  # sha256 of PREFILL_SRC when the prefill figures were taken
+BACKWARD_SRC = "exact_io_aware_41_b200/csrc/attn_bwd.cu"
+BACKWARD_SHA = "1b784b1041b43b92c5052df5fca0b12238063cacb7b463c8d0105884d6ee8957"
 NCU_TRAFFIC = {
-    # attn_fwd_kernel: 337.62 MB read + 49.63 MB written
-    synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 387_250_944.0),
-    # attn_fwd_kernel: 122.96 MB read + 9.71 MB written
-    synth.CAUSAL_2K.name: (PREFILL_SRC, PREFILL_SHA, 132_674_304.0),
-    # attn_fwd_kernel: 210.23 MB read + 47.78 MB written
-    synth.LONG_8K_CAUSAL.name: (PREFILL_SRC, PREFILL_SHA, 258_014_208.0),
-    # attn_fwd_kernel: 323.59 MB read + 101.11 MB written
-    synth.LONG_8K_GQA.name: (PREFILL_SRC, PREFILL_SHA, 424_704_000.0),
-    # attn_fwd_kernel: 369.60 MB read + 96.79 MB written
-    synth.LONG_8K_GQA_CAUSAL.name: (PREFILL_SRC, PREFILL_SHA, 466_393_344.0),
-    # attn_fwd_kernel: 50.45 MB read + 1.51 MB written
-    synth.SWEEP[0].name: (PREFILL_SRC, PREFILL_SHA, 51_952_128.0),
-    # attn_fwd_kernel: 116.12 MB read + 22.65 MB written
-    synth.SWEEP[1].name: (PREFILL_SRC, PREFILL_SHA, 138_769_664.0),
-    # attn_fwd_kernel: 330.37 MB read + 49.33 MB written
-    synth.SWEEP[2].name: (PREFILL_SRC, PREFILL_SHA, 379_698_432.0),
-    # attn_fwd_kernel: 689.65 MB read + 117.05 MB written
-    synth.SWEEP[3].name: (PREFILL_SRC, PREFILL_SHA, 806_694_400.0),
+    # attn_fwd_kernel<128>: 334.19 MB read + 49.36 MB written
+    synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 383_554_304.0),
+    # attn_fwd_kernel<128>: 122.57 MB read + 9.98 MB written
+    synth.CAUSAL_2K.name: (PREFILL_SRC, PREFILL_SHA, 132_545_792.0),
+    # attn_fwd_kernel<128>: 211.20 MB read + 47.87 MB written
+    synth.LONG_8K_CAUSAL.name: (PREFILL_SRC, PREFILL_SHA, 259_070_976.0),
+    # attn_fwd_kernel<128>: 322.24 MB read + 102.55 MB written
+    synth.LONG_8K_GQA.name: (PREFILL_SRC, PREFILL_SHA, 424_790_528.0),
+    # attn_fwd_kernel<128>: 368.13 MB read + 96.78 MB written
+    synth.LONG_8K_GQA_CAUSAL.name: (PREFILL_SRC, PREFILL_SHA, 464_904_192.0),
+    # attn_fwd_kernel<32>: 50.40 MB read + 1.45 MB written
+    synth.SWEEP[0].name: (PREFILL_SRC, PREFILL_SHA, 51_850_752.0),
+    # attn_fwd_kernel<64>: 118.28 MB read + 22.31 MB written
+    synth.SWEEP[1].name: (PREFILL_SRC, PREFILL_SHA, 140_589_568.0),
+    # attn_fwd_kernel<128>: 329.02 MB read + 47.94 MB written
+    synth.SWEEP[2].name: (PREFILL_SRC, PREFILL_SHA, 376_960_512.0),
+    # attn_fwd_kernel<256> on CTA pairs: 728.25 MB read + 116.16 MB written
+    synth.SWEEP[3].name: (PREFILL_SRC, PREFILL_SHA, 844_409_344.0),
+    # attn_fwd_kernel<128, 8-bit> on the long non-causal workload: 119.51 MB read + 41.89 MB written
+    "fp8 " + synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 161_400_064.0),
+    # attn_bwd_kernel on the causal N2048 workload: 417.13 MB read + 209.62 MB written
+    "backward " + synth.CAUSAL_2K.name: (BACKWARD_SRC, BACKWARD_SHA, 626_751_232.0),
     # decode_split_tc_kernel<128,4> (2123.81 MB read + 7.59 MB written) + decode_combine_kernel<128>
     # (4.29 MB read) on the full decode workload
     synth.DECODE.name: (DECODE_SRC, "eaf4990882bbcba5d723de8f5b505ab0c1520f88553cb35fa7ee6758aa501c3a", 2_135_693_824.0),
