@@ -401,7 +401,7 @@ def run_ours(args, world, rank, local, dist):
                   "prefill inputs; gates flush L2 (256 MiB write) before every launch",
         },
         "frac_of_nominal_bf16": pf_tflops_1 / NOMINAL_BF16_TFLOPS,
-        "roofline": {"bound": "tensor", "kernel": "attn::attn_fwd_kernel<128, false>",
+        "roofline": {"bound": "tensor", "kernel": "attn::attn_fwd_kernel<128, false, false>",
                      "achieved": pf_tflops_1, "peak": meas_tf, "unit": "TFLOP/s", "frac": pf_tflops_1 / meas_tf,
                      "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
                      "traffic": ncu_traffic(P.name), "traffic_source": "ncu dram__bytes_read.sum + "
@@ -463,7 +463,7 @@ def time_prefill(lib, w, dev, stream, peaks, reps=20, warm=5):
     tf = w.flops / (med * 1e-3) / 1e12
     pk = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
     return {"ms": med, "tflops": tf, "frac_of_measured": tf / pk, "frac_of_nominal": tf / NOMINAL_BF16_TFLOPS,
-            "roofline": {"bound": "tensor", "kernel": f"attn::attn_fwd_kernel<{w.d}, false>", "achieved": tf, "peak": pk,
+            "roofline": {"bound": "tensor", "kernel": f"attn::attn_fwd_kernel<{w.d}, false, {'true' if w.d == 256 else 'false'}>", "achieved": tf, "peak": pk,
                          "unit": "TFLOP/s", "frac": tf / pk, "traffic": ncu_traffic(w.name),
                          "algorithmic_bytes": prefill_bytes(w)}}
 
@@ -515,7 +515,7 @@ def time_prefill_fp8(lib, w, dev, stream, peaks, reps=20, warm=5):
     tf = w.flops / (med * 1e-3) / 1e12
     pk = 2.0 * peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
     return {"ms": med, "tflops": tf, "dtype": "e4m3 operands, fp32 accumulate",
-            "roofline": {"bound": "tensor", "kernel": "attn::attn_fwd_kernel<128, true>", "achieved": tf, "peak": pk,
+            "roofline": {"bound": "tensor", "kernel": "attn::attn_fwd_kernel<128, true, false>", "achieved": tf, "peak": pk,
                          "unit": "TFLOP/s", "frac": tf / pk, "peak_source": "2 x bf16 peak (nominal fp8/bf16 ratio)",
                          "traffic": ncu_traffic("fp8 " + w.name)}}
 

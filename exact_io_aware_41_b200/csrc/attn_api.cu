@@ -361,7 +361,7 @@ const char* attn_status_string(attn_status_t s) {
 
 const char* attn_kernel_name(int which) {
   switch (which) {
-    case 0: return "attn::attn_fwd_kernel<D, F8>";
+    case 0: return "attn::attn_fwd_kernel<D, F8, PAIR>";
     case 1: return "attn::decode_split_tc_kernel<D,G> (d <= 128), attn::decode_split_kernel<D,G> (d = 256)";
     case 2: return "attn::decode_combine_kernel<D>";
     case 3: return "attn::attn_bwd_pre_kernel, attn::attn_bwd_kernel, attn::attn_bwd_post_kernel";
