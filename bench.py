@@ -48,7 +48,7 @@ PREFILL_SRC = "exact_io_aware_41_b200/csrc/attn_fwd.cu"
 DECODE_SRC = "exact_io_aware_41_b200/csrc/attn_decode.cu"
 PREFILL_SHA = "0f72f8309b2d52a6219e56f70d6a4c9da93d023415cbe62689bc13f787aae103"  # sha256 of PREFILL_SRC when the prefill figures were taken
 BACKWARD_SRC = "exact_io_aware_41_b200/csrc/attn_bwd.cu"
-BACKWARD_SHA = "1b784b1041b43b92c5052df5fca0b12238063cacb7b463c8d0105884d6ee8957"
+BACKWARD_SHA = "0b5aa3b3ef65a549c286965423988f38526c5e3d1639a5e617c363b77a87fb73"
 NCU_TRAFFIC = {
     # attn_fwd_kernel<128>: 334.19 MB read + 49.36 MB written
     synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 383_554_304.0),
