@@ -13,12 +13,14 @@
 //   dS^T = P^T * (dP^T - D); P^T (bf16) over S^T, dS^T (bf16) over dP^T (each 32-query chunk's
 //   16 packed columns at the start of its own 32 score columns) and dS^T into shared memory
 //   dV += P^T dO     (A = P^T in TMEM, B = dO read MN-major)   -> columns [256, 384), whole unit
+//   dQ  = dS K       (A = dS from shared memory, M-major; B = K read MN-major) -> columns [0, 128)
 //   dK += dS^T Q     (A = dS^T in TMEM, B = Q read MN-major)   -> columns [384, 512), whole unit
-//   dQ  = dS K       (A = dS from shared memory, M-major; B = K read MN-major) -> columns [128, 256)
-//   the same warps stage dQ (thread = query row) in the step's Q / dO buffer, and the TMA unit adds
-//   it into an fp32 accumulator (cp.reduce.async.bulk.tensor ... add).
-// MMAs issued by one thread execute in issue order, so dQ may overwrite dS^T's columns after the dK
-// product that reads them, and the next step's S^T may overwrite P^T's after the dV product. Eight
+//   the same warps read dQ out (thread = query row) while dK runs, stage it in the step's Q / dO
+//   buffer, and the TMA unit adds it into an fp32 accumulator (cp.reduce.async.bulk.tensor ... add);
+//   the warps whose boxes go into the Q tile wait for dK, its last reader.
+// MMAs issued by one thread execute in issue order, so dQ may overwrite P^T's columns after the dV
+// product that reads them, and the next step's dP^T may overwrite dS^T's after the dK product; the
+// next step's S^T waits until dQ has been read out of its columns. Eight
 // warps (two per TMEM lane quadrant, 64 of the 128 columns each) do the elementwise work; Q, dO and
 // their LSE' and D rows are double-buffered so the next step's loads overlap this one. The unit ends
 // with dK (times scale) and dV stored as bf16.
@@ -53,8 +55,8 @@ constexpr int OFF_K = 0, OFF_V = TILE_BYTES, OFF_DS = 2 * TILE_BYTES;
 constexpr int OFF_Q0 = 3 * TILE_BYTES;        // stage s: Q at OFF_Q0 + 2s tiles, dO right after it
 constexpr int OFF_LSE0 = 7 * TILE_BYTES;      // stage s: LSE' at OFF_LSE0 + s * 1024, D 512 bytes later
 constexpr int OFF_BAR = OFF_LSE0 + 2 * 1024;
-// kv_full, q_full[2], q_empty[2], s_full, p_full, dq_full, dq_free, dkv_full
-constexpr int NBARS = 10;
+// kv_full, q_full[2], q_empty[2], s_full, p_full, dq_full, dq_free, dkv_full, dk_done
+constexpr int NBARS = 11;
 constexpr int SMEM_BYTES = OFF_BAR + NBARS * 8 + 16;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 }  // namespace bwd
@@ -117,6 +119,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
   uint64_t* dq_full = bars + 7;
   uint64_t* dq_free = bars + 8;
   uint64_t* dkv_full = bars + 9;
+  uint64_t* dk_done = bars + 10;  // one phase per step: the step's dK product (the last reader of Q) is done
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -143,6 +146,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
     mbar_init(dq_full, 1);
     mbar_init(dq_free, NSW);  // one arrival per softmax warp
     mbar_init(dkv_full, 1);
+    mbar_init(dk_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -217,19 +221,19 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
         ok = mbar_wait(&q_full[st], uint32_t((t >> 1) & 1), abort_flag, T);
         if (!ok) break;
         tc_fence_after();
-        // S^T = K Q^T into [0, 128): P^T of the previous step there was read by its dV product,
-        // issued earlier by this thread
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * CHUNK_BYTES + (kk % 4) * 32) >> 4;
-          umma_ss(tmem + S_COL, dK_k + off, dQ_k + off, idesc_kk, kk > 0 ? 1u : 0u);
-        }
-        // dP^T = V dO^T into [128, 256), once the previous step's dQ (there) has been read out
+        // S^T = K Q^T into [0, 128), once the previous step's dQ (there) has been read out
         if (t > 0) {
           ok = mbar_wait(dq_free, uint32_t((t - 1) & 1), abort_flag, T);
           if (!ok) break;
           tc_fence_after();
         }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * CHUNK_BYTES + (kk % 4) * 32) >> 4;
+          umma_ss(tmem + S_COL, dK_k + off, dQ_k + off, idesc_kk, kk > 0 ? 1u : 0u);
+        }
+        // dP^T = V dO^T into [128, 256): dS^T of the previous step there was read by its dK product,
+        // issued earlier by this thread
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * CHUNK_BYTES + (kk % 4) * 32) >> 4;
@@ -239,8 +243,8 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
         ok = mbar_wait(p_full, uint32_t(t & 1), abort_flag, T);
         if (!ok) break;
         tc_fence_after();
-        // over the step's 128 queries (k-steps of 16): dV += P^T dO, dK += dS^T Q, then dQ = dS K
-        // into [128, 256), after the dK product has read dS^T there
+        // over the step's 128 queries (k-steps of 16): dV += P^T dO, then dQ = dS K into [0, 128)
+        // (after the dV product has read P^T there), whose read-out overlaps dK += dS^T Q
         // A = P^T / dS^T: queries 16kk .. 16kk+15 are columns 8 (kk % 2) .. of chunk kk / 2, which
         // starts at column 32 (kk / 2)
 #pragma unroll
@@ -248,14 +252,15 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
           umma_ts(tmem + DV_COL, tmem + S_COL + 32 * (kk / 2) + 8 * (kk % 2),
                   dDO_mn + uint64_t((kk * 16 * 128) >> 4), idesc_tmn, (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_ss(tmem + S_COL, dDS_mn + uint64_t((kk * 16 * 128) >> 4), dK_mn + uint64_t((kk * 16 * 128) >> 4),
+                  idesc_mnmn, kk > 0 ? 1u : 0u);
+        umma_commit(dq_full);
+#pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
           umma_ts(tmem + DK_COL, tmem + DP_COL + 32 * (kk / 2) + 8 * (kk % 2),
                   dQ_mn + uint64_t((kk * 16 * 128) >> 4), idesc_tmn, (t > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          umma_ss(tmem + DP_COL, dDS_mn + uint64_t((kk * 16 * 128) >> 4), dK_mn + uint64_t((kk * 16 * 128) >> 4),
-                  idesc_mnmn, kk > 0 ? 1u : 0u);
-        umma_commit(dq_full);
+        umma_commit(dk_done);
         if (t == n_steps - 1) umma_commit(dkv_full);
       }
       if (!ok) {
@@ -352,20 +357,19 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
         bulk_wait_group_read0();
         mbar_arrive(&q_empty[(t - 1) & 1]);
       }
-      // dQ of this step (thread = query row q0 + row, this warp's 64 of the d columns): once every
-      // product of the step is done, read it from TMEM and release those columns, then stage it as
-      // two 32 x 32 fp32 boxes (128-byte rows, swizzled like the tensor map) in this step's Q / dO
-      // buffer, which no product reads any more, and let the TMA unit add the boxes into the fp32
-      // accumulator. The buffer goes back to the producer once the TMA has read it (checked one
-      // step later, above).
+      // dQ of this step (thread = query row q0 + row, this warp's 64 of the d columns): once the dQ
+      // product is done, read it from TMEM and release those columns, then stage it as two 32 x 32
+      // fp32 boxes (128-byte rows, swizzled like the tensor map) in this step's Q / dO buffer, and
+      // let the TMA unit add the boxes into the fp32 accumulator. The buffer goes back to the
+      // producer once the TMA has read it (checked one step later, above).
       if (!wait_warp(dq_full, uint32_t(t & 1))) {
         ok = false;
         break;
       }
       tc_fence_after();
       uint32_t o[2][32];
-      tmem_ld32(lane_addr + DP_COL + (2 * hf) * 32, o[0]);
-      tmem_ld32(lane_addr + DP_COL + (2 * hf + 1) * 32, o[1]);
+      tmem_ld32(lane_addr + S_COL + (2 * hf) * 32, o[0]);
+      tmem_ld32(lane_addr + S_COL + (2 * hf + 1) * 32, o[1]);
       tmem_ld_wait();
       tmem_reg_fence32(o[0]);
       tmem_reg_fence32(o[1]);
@@ -373,6 +377,12 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
       const int row0 = q0 + wq * 32;  // first query row of this warp's boxes
+      // warps 8-11 stage into the step's dO tile, read last by dV (done); warps 4-7 into its Q tile,
+      // read last by dK, which runs after dQ: those wait for it
+      if (hf == 0 && !wait_warp(dk_done, uint32_t(t & 1))) {
+        ok = false;
+        break;
+      }
       uint8_t* box = smem + OFF_Q0 + 2 * (t & 1) * TILE_BYTES + (warp - 4) * 8192;
 #pragma unroll
       for (int cx = 0; cx < 2; ++cx)
