@@ -42,7 +42,12 @@ constexpr int BM = 128;                       // query rows per step
 constexpr int BN = 128;                       // keys per CTA
 constexpr int CHUNK_BYTES = 128 * 128;        // 64-column chunk of a 128-row tile (128-byte rows)
 constexpr int TILE_BYTES = 2 * CHUNK_BYTES;   // 128 x 128 bf16
-constexpr int NSW = 8;                        // softmax / epilogue warps: two per TMEM lane quadrant
+#ifndef ATTN_BWD_WARPS
+#define ATTN_BWD_WARPS 8
+#endif
+constexpr int NSW = ATTN_BWD_WARPS;           // softmax / epilogue warps: NSW / 4 per TMEM lane quadrant
+constexpr int CPW = 16 / NSW;                 // 32-column chunks of a 128-column tile per warp
+static_assert(NSW == 8 || NSW == 16, "8 or 16 elementwise warps");
 constexpr int THREADS = 128 + 32 * NSW;
 constexpr int TMEM_COLS = 512;
 constexpr int S_COL = 0, DP_COL = 128, DV_COL = 256, DK_COL = 384;
@@ -274,7 +279,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
   } else if (warp >= 4) {
     // ========================= softmax / dQ / dK dV epilogue warps =========================
     const int wq = warp & 3;
-    const int hf = (warp - 4) >> 2;   // which 64 of the 128 columns this warp covers
+    const int cw = (warp - 4) >> 2;   // which CPW x 32 of the 128 columns this warp covers
     const int row = wq * 32 + lane;   // TMEM lane: key row (softmax, dK dV) or query row (dQ)
     const uint32_t lane_addr = tmem + (uint32_t(wq * 32) << 16);
     const float c = args.scale_log2;
@@ -297,8 +302,8 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
       tc_fence_after();
       const int q0 = qt * BM;
 #pragma unroll 1
-      for (int cx = 0; cx < 2; ++cx) {  // 32 query columns at a time, this warp's 64
-        const int cc = 2 * hf + cx;
+      for (int cx = 0; cx < CPW; ++cx) {  // 32 query columns at a time, this warp's CPW x 32
+        const int cc = CPW * cw + cx;
         uint32_t sv[32], dpv[32];
         tmem_ld32(lane_addr + S_COL + cc * 32, sv);
         tmem_ld32(lane_addr + DP_COL + cc * 32, dpv);
@@ -367,25 +372,26 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
         break;
       }
       tc_fence_after();
-      uint32_t o[2][32];
-      tmem_ld32(lane_addr + S_COL + (2 * hf) * 32, o[0]);
-      tmem_ld32(lane_addr + S_COL + (2 * hf + 1) * 32, o[1]);
+      uint32_t o[CPW][32];
+#pragma unroll
+      for (int cx = 0; cx < CPW; ++cx) tmem_ld32(lane_addr + S_COL + (CPW * cw + cx) * 32, o[cx]);
       tmem_ld_wait();
-      tmem_reg_fence32(o[0]);
-      tmem_reg_fence32(o[1]);
+#pragma unroll
+      for (int cx = 0; cx < CPW; ++cx) tmem_reg_fence32(o[cx]);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
       const int row0 = q0 + wq * 32;  // first query row of this warp's boxes
-      // warps 8-11 stage into the step's dO tile, read last by dV (done); warps 4-7 into its Q tile,
-      // read last by dK, which runs after dQ: those wait for it
-      if (hf == 0 && !wait_warp(dk_done, uint32_t(t & 1))) {
+      // the second half of the warps stage into the step's dO tile, read last by dV (done); the first
+      // half into its Q tile, read last by dK, which runs after dQ: those wait for it
+      const int box_off = (warp - 4) * CPW * 4096;
+      if (box_off < TILE_BYTES && !wait_warp(dk_done, uint32_t(t & 1))) {
         ok = false;
         break;
       }
-      uint8_t* box = smem + OFF_Q0 + 2 * (t & 1) * TILE_BYTES + (warp - 4) * 8192;
+      uint8_t* box = smem + OFF_Q0 + 2 * (t & 1) * TILE_BYTES + box_off;
 #pragma unroll
-      for (int cx = 0; cx < 2; ++cx)
+      for (int cx = 0; cx < CPW; ++cx)
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const uint32_t a = smem_u32(box + cx * 4096) + lane * 128 + ((u ^ (lane & 7)) << 4);
@@ -396,8 +402,8 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0 && row0 < args.Nq) {  // rows past Nq are clipped by the TMA unit
-        tma_reduce_add_4d(&tmDQ, box, (2 * hf) * 32, h, row0, b);
-        tma_reduce_add_4d(&tmDQ, box + 4096, (2 * hf + 1) * 32, h, row0, b);
+#pragma unroll
+        for (int cx = 0; cx < CPW; ++cx) tma_reduce_add_4d(&tmDQ, box + cx * 4096, (CPW * cw + cx) * 32, h, row0, b);
         bulk_commit_group();
       }
       __syncwarp();
@@ -407,8 +413,8 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
     if (key_ok && n_steps == 0) {
       for (int which = 0; which < 2; ++which) {
         uint4* dz = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(which ? args.dv : args.dk) +
-                                             ((size_t(b) * args.Nkv + key) * args.Hkv + g) * D + 64 * hf);
-        for (int v4 = 0; v4 < 8; ++v4) dz[v4] = make_uint4(0, 0, 0, 0);
+                                             ((size_t(b) * args.Nkv + key) * args.Hkv + g) * D + 32 * CPW * cw);
+        for (int v4 = 0; v4 < 4 * CPW; ++v4) dz[v4] = make_uint4(0, 0, 0, 0);
       }
     }
     if (n_steps > 0 && ok && wait_warp(dkv_full, 0)) {
@@ -419,8 +425,8 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
         __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(which == 0 ? args.dk : args.dv) +
                              ((size_t(b) * args.Nkv + (key_ok ? key : 0)) * args.Hkv + g) * D;
 #pragma unroll 1
-        for (int cx = 0; cx < 2; ++cx) {
-          const int cc = 2 * hf + cx;
+        for (int cx = 0; cx < CPW; ++cx) {
+          const int cc = CPW * cw + cx;
           uint32_t o[32];
           tmem_ld32(lane_addr + (which == 0 ? DK_COL : DV_COL) + cc * 32, o);
           tmem_ld_wait();

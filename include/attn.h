@@ -63,7 +63,10 @@ typedef enum {
  * memory, assigned to launches round robin and returned to zero by each launch's last CTA. Launches
  * on one stream never overlap, and launches on different streams are safe as long as fewer than
  * 256 later prefill launches on that device start before an earlier one finishes (a launch held
- * back behind a cross-stream wait while 256 others run past it would share a counter).
+ * back behind a cross-stream wait while 256 others run past it would share a counter). d = 256
+ * launches clusters of two CTAs (2-SM tensor-core products) with a fixed share of the work per
+ * cluster and uses no claim counter; it needs a device and context where clusters of two can be
+ * resident (ATTN_ERR_CUDA otherwise).
  */
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                        int Hkv, int Nq, int Nkv, int d, float scale, int causal, cudaStream_t stream);
