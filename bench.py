@@ -46,32 +46,32 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 # that file changes, the figure is stale and the bench line reports null until it is measured again.
 PREFILL_SRC = "exact_io_aware_41_b200/csrc/attn_fwd.cu"
 DECODE_SRC = "exact_io_aware_41_b200/csrc/attn_decode.cu"
-PREFILL_SHA = "0f72f8309b2d52a6219e56f70d6a4c9da93d023415cbe62689bc13f787aae103"  # sha256 of PREFILL_SRC when the prefill figures were taken
+PREFILL_SHA = "529761043c67af8eaf37eebba58db85453f3ffe41351f2bd98792fbc3489d47f"  # sha256 of PREFILL_SRC when the prefill figures were taken
 BACKWARD_SRC = "exact_io_aware_41_b200/csrc/attn_bwd.cu"
-BACKWARD_SHA = "0b5aa3b3ef65a549c286965423988f38526c5e3d1639a5e617c363b77a87fb73"
+BACKWARD_SHA = "5c63776922444124f623b4467ac34ebc79ef7a21ba9ed3d21768ca781d351b6a"
 NCU_TRAFFIC = {
-    # attn_fwd_kernel<128>: 334.19 MB read + 49.36 MB written
-    synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 383_554_304.0),
-    # attn_fwd_kernel<128>: 122.57 MB read + 9.98 MB written
-    synth.CAUSAL_2K.name: (PREFILL_SRC, PREFILL_SHA, 132_545_792.0),
-    # attn_fwd_kernel<128>: 211.20 MB read + 47.87 MB written
-    synth.LONG_8K_CAUSAL.name: (PREFILL_SRC, PREFILL_SHA, 259_070_976.0),
-    # attn_fwd_kernel<128>: 322.24 MB read + 102.55 MB written
-    synth.LONG_8K_GQA.name: (PREFILL_SRC, PREFILL_SHA, 424_790_528.0),
-    # attn_fwd_kernel<128>: 368.13 MB read + 96.78 MB written
-    synth.LONG_8K_GQA_CAUSAL.name: (PREFILL_SRC, PREFILL_SHA, 464_904_192.0),
-    # attn_fwd_kernel<32>: 50.40 MB read + 1.45 MB written
-    synth.SWEEP[0].name: (PREFILL_SRC, PREFILL_SHA, 51_850_752.0),
-    # attn_fwd_kernel<64>: 118.28 MB read + 22.31 MB written
-    synth.SWEEP[1].name: (PREFILL_SRC, PREFILL_SHA, 140_589_568.0),
-    # attn_fwd_kernel<128>: 329.02 MB read + 47.94 MB written
-    synth.SWEEP[2].name: (PREFILL_SRC, PREFILL_SHA, 376_960_512.0),
-    # attn_fwd_kernel<256> on CTA pairs: 728.25 MB read + 116.16 MB written
-    synth.SWEEP[3].name: (PREFILL_SRC, PREFILL_SHA, 844_409_344.0),
-    # attn_fwd_kernel<128, 8-bit> on the long non-causal workload: 119.51 MB read + 41.89 MB written
-    "fp8 " + synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 161_400_064.0),
-    # attn_bwd_kernel on the causal N2048 workload: 417.13 MB read + 209.62 MB written
-    "backward " + synth.CAUSAL_2K.name: (BACKWARD_SRC, BACKWARD_SHA, 626_751_232.0),
+    # attn_fwd_kernel<128>: 325.10 MB read + 52.82 MB written
+    synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 377_920_512.0),
+    # attn_fwd_kernel<128>: 126.51 MB read + 11.05 MB written
+    synth.CAUSAL_2K.name: (PREFILL_SRC, PREFILL_SHA, 137_565_952.0),
+    # attn_fwd_kernel<128>: 211.65 MB read + 49.96 MB written
+    synth.LONG_8K_CAUSAL.name: (PREFILL_SRC, PREFILL_SHA, 261_611_264.0),
+    # attn_fwd_kernel<128>: 355.00 MB read + 107.24 MB written
+    synth.LONG_8K_GQA.name: (PREFILL_SRC, PREFILL_SHA, 462_240_256.0),
+    # attn_fwd_kernel<128>: 365.01 MB read + 101.65 MB written
+    synth.LONG_8K_GQA_CAUSAL.name: (PREFILL_SRC, PREFILL_SHA, 466_659_840.0),
+    # attn_fwd_kernel<32>: 50.49 MB read + 1.45 MB written
+    synth.SWEEP[0].name: (PREFILL_SRC, PREFILL_SHA, 51_934_976.0),
+    # attn_fwd_kernel<64>: 117.44 MB read + 22.53 MB written
+    synth.SWEEP[1].name: (PREFILL_SRC, PREFILL_SHA, 139_966_464.0),
+    # attn_fwd_kernel<128>: 331.34 MB read + 51.31 MB written
+    synth.SWEEP[2].name: (PREFILL_SRC, PREFILL_SHA, 382_650_368.0),
+    # attn_fwd_kernel<256> on CTA pairs: 720.36 MB read + 119.08 MB written
+    synth.SWEEP[3].name: (PREFILL_SRC, PREFILL_SHA, 839_432_448.0),
+    # attn_fwd_kernel<128, 8-bit> on the long non-causal workload: 131.08 MB read + 42.57 MB written
+    "fp8 " + synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 173_644_032.0),
+    # attn_bwd_kernel on the causal N2048 workload: 427.31 MB read + 214.98 MB written
+    "backward " + synth.CAUSAL_2K.name: (BACKWARD_SRC, BACKWARD_SHA, 642_291_968.0),
     # decode_split_tc_kernel<128,4> (2123.81 MB read + 7.59 MB written) + decode_combine_kernel<128>
     # (4.29 MB read) on the full decode workload
     synth.DECODE.name: (DECODE_SRC, "eaf4990882bbcba5d723de8f5b505ab0c1520f88553cb35fa7ee6758aa501c3a", 2_135_693_824.0),
