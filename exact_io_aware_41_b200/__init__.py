@@ -38,6 +38,7 @@ SIGNATURES = {
     "attn_status_string": (ctypes.c_char_p, [_I]),
     "attn_kernel_name": (ctypes.c_char_p, [_I]),
     "attn_selftest_bounded_wait": (_I, [ctypes.c_uint, _P]),
+    "attn_selftest_pair_wait": (_I, [ctypes.c_uint, _I, _P]),
     "attn_selftest_exp2_poly": (_I, [_P, _P, _I, _P]),
     "attn_fp8_quantize": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "attn_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
@@ -223,6 +224,11 @@ def attn_get_last_error() -> int:
 
 def attn_selftest_bounded_wait(limit_us: int, stream=None) -> None:
     _check("attn_selftest_bounded_wait", lib_handle().attn_selftest_bounded_wait(int(limit_us), _stream(stream)))
+
+
+def attn_selftest_pair_wait(limit_us: int, cross_arrive: bool, stream=None) -> None:
+    _check("attn_selftest_pair_wait",
+           lib_handle().attn_selftest_pair_wait(int(limit_us), 1 if cross_arrive else 0, _stream(stream)))
 
 
 def attn_selftest_exp2_poly(x, out=None, stream=None):

@@ -23,6 +23,29 @@ __global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns) {
   __syncthreads();
 }
 
+// A cluster of two CTAs: each CTA's thread 0 waits (bounded, cluster-scope acquire) on its own
+// mbarrier, after arriving on the other CTA's through its shared::cluster address when cross_arrive
+// is set (the hand-off the prefill's CTA pairs use); without it nothing completes either barrier and
+// both waits run out. Both CTAs meet at the cluster barrier before exiting.
+__global__ void pair_wait_selftest_kernel(unsigned long long limit_ns, int cross_arrive) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t rank = cluster_ctarank();
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  cluster_sync();
+  if (threadIdx.x == 0) {
+    if (cross_arrive) mbar_arrive_cluster(mapa_shared(&bar, rank ^ 1u));
+    mbar_wait_cluster(&bar, 0, &abort_flag, limit_ns);
+  }
+  __syncthreads();
+  cluster_sync();
+}
+
 // 2^x through the FMA-pipe polynomial (exp2_poly2), two values per thread, for checking it against
 // the exact function.
 __global__ void exp2_poly_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
@@ -373,6 +396,26 @@ attn_status_t attn_selftest_bounded_wait(unsigned int limit_us, cudaStream_t str
   if (limit_us == 0 || limit_us > 10000000u) return ATTN_ERR_INVALID_ARG;
   bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(1000ull * limit_us);
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
+}
+
+attn_status_t attn_selftest_pair_wait(unsigned int limit_us, int cross_arrive, cudaStream_t stream) {
+  if (limit_us == 0 || limit_us > 10000000u || (cross_arrive != 0 && cross_arrive != 1)) return ATTN_ERR_INVALID_ARG;
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  lc.gridDim = dim3(2);
+  lc.blockDim = dim3(32);
+  lc.stream = stream;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  if (cudaLaunchKernelEx(&lc, pair_wait_selftest_kernel, 1000ull * limit_us, cross_arrive) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
 }
 
 attn_status_t attn_selftest_exp2_poly(const float* x, float* y, int n, cudaStream_t stream) {

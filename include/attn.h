@@ -232,6 +232,16 @@ const char* attn_kernel_name(int which);
 attn_status_t attn_selftest_bounded_wait(unsigned int limit_us, cudaStream_t stream);
 
 /*
+ * Test hook for the waits between the two CTAs of a cluster (the d = 256 prefill's CTA pairs):
+ * launches one cluster of two CTAs; in each, one thread waits with the given limit (microseconds) on
+ * an mbarrier of its own CTA. cross_arrive = 1: each CTA first arrives on the other's barrier through
+ * its cluster address, both waits complete and attn_get_last_error() stays ATTN_OK; cross_arrive =
+ * 0: nothing arrives, both waits run out and it reports ATTN_ERR_TIMEOUT. Nothing faults or hangs.
+ * ATTN_ERR_INVALID_ARG for limit_us outside [1, 10^7] or cross_arrive other than 0 or 1.
+ */
+attn_status_t attn_selftest_pair_wait(unsigned int limit_us, int cross_arrive, cudaStream_t stream);
+
+/*
  * Test hook for the FMA-pipe exponential (Cody-Waite range reduction and a degree-3 polynomial;
  * the "emulated exponentials" the FlashAttention generation comparison record describes for
  * FA-4). The prefill kernels can evaluate part of their exponentials with it (a build option, off

@@ -102,6 +102,8 @@ def test_argument_errors_are_reported_before_any_launch(raw):
     assert lib.attn_decode_combine(p, p, 4, 4, 96, p, p, None) == pkg.ATTN_ERR_UNSUPPORTED
     assert lib.attn_decode_combine(p, p, 4, 25601, 128, p, p, None) == pkg.ATTN_ERR_UNSUPPORTED
     assert lib.attn_selftest_bounded_wait(0, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert lib.attn_selftest_pair_wait(0, 1, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert lib.attn_selftest_pair_wait(1000, 2, None) == pkg.ATTN_ERR_INVALID_ARG
     assert lib.attn_selftest_exp2_poly(None, p, 4, None) == pkg.ATTN_ERR_INVALID_ARG
     assert lib.attn_selftest_exp2_poly(p, p, 0, None) == pkg.ATTN_ERR_INVALID_ARG
     assert lib.attn_selftest_exp2_poly(p + 2, p, 4, None) == pkg.ATTN_ERR_INVALID_ARG

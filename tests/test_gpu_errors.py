@@ -17,6 +17,20 @@ def test_bounded_wait_times_out_and_reports(lib):
     assert float(x.sum()) == 1024.0
 
 
+def test_cluster_pair_waits_complete_or_time_out(lib):
+    import torch
+
+    assert lib.attn_get_last_error() == lib.ATTN_OK
+    lib.attn_selftest_pair_wait(2000000, True)  # each CTA arrives on the other's barrier: no timeout
+    torch.cuda.synchronize()
+    assert lib.attn_get_last_error() == lib.ATTN_OK
+    lib.attn_selftest_pair_wait(2000, False)  # nothing arrives: both 2 ms waits run out
+    torch.cuda.synchronize()
+    assert lib.attn_get_last_error() == lib.ATTN_ERR_TIMEOUT
+    x = torch.ones(1024, device="cuda")
+    assert float(x.sum()) == 1024.0
+
+
 def test_argument_errors_raise(lib):
     import torch
 
