@@ -320,19 +320,23 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
           const float4 l4 = *reinterpret_cast<const float4*>(s_lse + cc * 32 + 4 * i4);
           const float4 d4 = *reinterpret_cast<const float4*>(s_dd + cc * 32 + 4 * i4);
           const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-          float p4[4], ds4[4];
+          // pairs of query columns on the packed FMA pipe (the same roundings as the scalar forms)
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int qi = cc * 32 + 4 * i4 + u;
-            float p = ex2(fmaf(__uint_as_float(sv[4 * i4 + u]), c, -lv[u]));
-            if (need_mask && !(key_ok && (!args.causal || key <= q0 + qi + diag))) p = 0.f;
-            p4[u] = p;
-            ds4[u] = p * (__uint_as_float(dpv[4 * i4 + u]) - dv4[u]);
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int u = 2 * h2, qi = cc * 32 + 4 * i4 + u;
+            const float2 x = ffma2(make_float2(__uint_as_float(sv[4 * i4 + u]), __uint_as_float(sv[4 * i4 + u + 1])),
+                                   make_float2(c, c), make_float2(-lv[u], -lv[u + 1]));
+            float2 p = make_float2(ex2(x.x), ex2(x.y));
+            if (need_mask) {
+              if (!(key_ok && (!args.causal || key <= q0 + qi + diag))) p.x = 0.f;
+              if (!(key_ok && (!args.causal || key <= q0 + qi + 1 + diag))) p.y = 0.f;
+            }
+            const float2 ds = fmul2(p, fadd2(make_float2(__uint_as_float(dpv[4 * i4 + u]),
+                                                         __uint_as_float(dpv[4 * i4 + u + 1])),
+                                             make_float2(-dv4[u], -dv4[u + 1])));
+            pk[2 * i4 + h2] = pack_bf16x2(p.x, p.y);
+            dk2[2 * i4 + h2] = pack_bf16x2(ds.x, ds.y);
           }
-          pk[2 * i4] = pack_bf16x2(p4[0], p4[1]);
-          pk[2 * i4 + 1] = pack_bf16x2(p4[2], p4[3]);
-          dk2[2 * i4] = pack_bf16x2(ds4[0], ds4[1]);
-          dk2[2 * i4 + 1] = pack_bf16x2(ds4[2], ds4[3]);
         }
         // P^T over S^T and dS^T over dP^T, bf16 pairs: the chunk's 16 columns go to the first 16 of
         // its own 32 score columns (just read), so no warp writes where the other still reads
