@@ -48,7 +48,7 @@ PREFILL_SRC = "exact_io_aware_41_b200/csrc/attn_fwd.cu"
 DECODE_SRC = "exact_io_aware_41_b200/csrc/attn_decode.cu"
 PREFILL_SHA = "529761043c67af8eaf37eebba58db85453f3ffe41351f2bd98792fbc3489d47f"  # sha256 of PREFILL_SRC when the prefill figures were taken
 BACKWARD_SRC = "exact_io_aware_41_b200/csrc/attn_bwd.cu"
-BACKWARD_SHA = "5c63776922444124f623b4467ac34ebc79ef7a21ba9ed3d21768ca781d351b6a"
+BACKWARD_SHA = "1fa40e25e689587d0be9a5542e661af53df25f4de7451151ba7f11e6421093dc"
 NCU_TRAFFIC = {
     # attn_fwd_kernel<128>: 325.10 MB read + 52.82 MB written
     synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 377_920_512.0),
@@ -70,8 +70,8 @@ NCU_TRAFFIC = {
     synth.SWEEP[3].name: (PREFILL_SRC, PREFILL_SHA, 839_432_448.0),
     # attn_fwd_kernel<128, 8-bit> on the long non-causal workload: 131.08 MB read + 42.57 MB written
     "fp8 " + synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 173_644_032.0),
-    # attn_bwd_kernel on the causal N2048 workload: 427.31 MB read + 214.98 MB written
-    "backward " + synth.CAUSAL_2K.name: (BACKWARD_SRC, BACKWARD_SHA, 642_291_968.0),
+    # attn_bwd_kernel on the causal N2048 workload: 425.18 MB read + 215.12 MB written
+    "backward " + synth.CAUSAL_2K.name: (BACKWARD_SRC, BACKWARD_SHA, 640_295_936.0),
     # decode_split_tc_kernel<128,4> (2123.81 MB read + 7.59 MB written) + decode_combine_kernel<128>
     # (4.29 MB read) on the full decode workload
     synth.DECODE.name: (DECODE_SRC, "eaf4990882bbcba5d723de8f5b505ab0c1520f88553cb35fa7ee6758aa501c3a", 2_135_693_824.0),
