@@ -1,9 +1,10 @@
 // Prefill forward for sm_100a: O = softmax(scale * Q K^T) V and LSE, tile by tile.
 //
-// Work decomposition: a unit is (batch b, query head h, block of NQT query tiles of 128 rows). The
-// grid is persistent (one CTA per SM); each CTA claims units from a per-launch atomic counter.
-// Units are numbered by L2 head group and, inside a group, heaviest first (longest-processing-time
-// order for causal masks). Query-block parallelism follows the "FlashAttention evolution" article,
+// Work decomposition: a unit is (batch b, query head h, block of NQT query tiles of 128 rows; at
+// d = 256 one tile in each CTA of a pair). The grid is persistent (one CTA per SM); each CTA claims
+// units from a per-launch atomic counter (CTA pairs take fixed shares instead). Units are numbered
+// by L2 head group and, inside a group, heaviest first (longest-processing-time order for causal
+// masks). Query-block parallelism follows the "FlashAttention evolution" article,
 // section 3; LPT ordering the FlashAttention generation comparison record, "Workarounds" (FA-4).
 //
 // Roles inside a CTA (warp specialisation, evolution article section 4, rebuilt on sm_100a):

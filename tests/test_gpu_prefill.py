@@ -77,6 +77,11 @@ def test_head_dim_256_cta_pairs(lib):
     _run_small(lib, 4501, 1, 2, 2, 130, 130, 256, True)
     _run_small(lib, 4502, 1, 2, 2, 1, 193, 256, False)
     _run_small(lib, 4503, 2, 8, 4, 1300, 1300, 256, True, scale=0.125)
+    # one key (the second CTA's half of the only K tile lies wholly past the end), one query row,
+    # and a causal square smaller than a tile
+    _run_small(lib, 4504, 1, 2, 2, 300, 1, 256, False)
+    _run_small(lib, 4505, 1, 2, 1, 1, 1, 256, True)
+    _run_small(lib, 4506, 2, 2, 2, 5, 5, 256, True)
 
 
 @pytest.mark.parametrize("d", [32, 64])
