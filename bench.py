@@ -46,30 +46,30 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 # that file changes, the figure is stale and the bench line reports null until it is measured again.
 PREFILL_SRC = "exact_io_aware_41_b200/csrc/attn_fwd.cu"
 DECODE_SRC = "exact_io_aware_41_b200/csrc/attn_decode.cu"
-PREFILL_SHA = "529761043c67af8eaf37eebba58db85453f3ffe41351f2bd98792fbc3489d47f"  # sha256 of PREFILL_SRC when the prefill figures were taken
+PREFILL_SHA = "63b6180f1f6afe9c54d540d7fed48ed998708272751ad149f087cb68eb2d9625"  # sha256 of PREFILL_SRC when the prefill figures were taken
 BACKWARD_SRC = "exact_io_aware_41_b200/csrc/attn_bwd.cu"
 BACKWARD_SHA = "1fa40e25e689587d0be9a5542e661af53df25f4de7451151ba7f11e6421093dc"
 NCU_TRAFFIC = {
-    # attn_fwd_kernel<128>: 325.10 MB read + 52.82 MB written
-    synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 377_920_512.0),
-    # attn_fwd_kernel<128>: 126.51 MB read + 11.05 MB written
-    synth.CAUSAL_2K.name: (PREFILL_SRC, PREFILL_SHA, 137_565_952.0),
-    # attn_fwd_kernel<128>: 211.65 MB read + 49.96 MB written
-    synth.LONG_8K_CAUSAL.name: (PREFILL_SRC, PREFILL_SHA, 261_611_264.0),
-    # attn_fwd_kernel<128>: 355.00 MB read + 107.24 MB written
-    synth.LONG_8K_GQA.name: (PREFILL_SRC, PREFILL_SHA, 462_240_256.0),
-    # attn_fwd_kernel<128>: 365.01 MB read + 101.65 MB written
-    synth.LONG_8K_GQA_CAUSAL.name: (PREFILL_SRC, PREFILL_SHA, 466_659_840.0),
-    # attn_fwd_kernel<32>: 50.49 MB read + 1.45 MB written
-    synth.SWEEP[0].name: (PREFILL_SRC, PREFILL_SHA, 51_934_976.0),
-    # attn_fwd_kernel<64>: 117.44 MB read + 22.53 MB written
-    synth.SWEEP[1].name: (PREFILL_SRC, PREFILL_SHA, 139_966_464.0),
-    # attn_fwd_kernel<128>: 331.34 MB read + 51.31 MB written
-    synth.SWEEP[2].name: (PREFILL_SRC, PREFILL_SHA, 382_650_368.0),
-    # attn_fwd_kernel<256> on CTA pairs: 720.36 MB read + 119.08 MB written
-    synth.SWEEP[3].name: (PREFILL_SRC, PREFILL_SHA, 839_432_448.0),
-    # attn_fwd_kernel<128, 8-bit> on the long non-causal workload: 131.08 MB read + 42.57 MB written
-    "fp8 " + synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 173_644_032.0),
+    # attn_fwd_kernel<128>: 350.77 MB read + 52.83 MB written
+    synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 403_600_640.0),
+    # attn_fwd_kernel<128>: 128.36 MB read + 13.21 MB written
+    synth.CAUSAL_2K.name: (PREFILL_SRC, PREFILL_SHA, 141_571_328.0),
+    # attn_fwd_kernel<128>: 213.84 MB read + 50.57 MB written
+    synth.LONG_8K_CAUSAL.name: (PREFILL_SRC, PREFILL_SHA, 264_412_160.0),
+    # attn_fwd_kernel<128>: 369.63 MB read + 106.79 MB written
+    synth.LONG_8K_GQA.name: (PREFILL_SRC, PREFILL_SHA, 476_417_024.0),
+    # attn_fwd_kernel<128>: 373.41 MB read + 101.96 MB written
+    synth.LONG_8K_GQA_CAUSAL.name: (PREFILL_SRC, PREFILL_SHA, 475_375_616.0),
+    # attn_fwd_kernel<32>: 50.40 MB read + 1.50 MB written
+    synth.SWEEP[0].name: (PREFILL_SRC, PREFILL_SHA, 51_898_624.0),
+    # attn_fwd_kernel<64>: 114.14 MB read + 22.27 MB written
+    synth.SWEEP[1].name: (PREFILL_SRC, PREFILL_SHA, 136_412_928.0),
+    # attn_fwd_kernel<128>: 345.82 MB read + 53.71 MB written
+    synth.SWEEP[2].name: (PREFILL_SRC, PREFILL_SHA, 399_529_984.0),
+    # attn_fwd_kernel<256> on CTA pairs: 743.03 MB read + 118.83 MB written
+    synth.SWEEP[3].name: (PREFILL_SRC, PREFILL_SHA, 861_856_512.0),
+    # attn_fwd_kernel<128, 8-bit> on the long non-causal workload: 138.46 MB read + 42.28 MB written
+    "fp8 " + synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 180_734_720.0),
     # attn_bwd_kernel on the causal N2048 workload: 425.18 MB read + 215.12 MB written
     "backward " + synth.CAUSAL_2K.name: (BACKWARD_SRC, BACKWARD_SHA, 640_295_936.0),
     # decode_split_tc_kernel<128,4> (2123.81 MB read + 7.59 MB written) + decode_combine_kernel<128>
