@@ -15,9 +15,10 @@
 //   dV += P^T dO     (A = P^T in TMEM, B = dO read MN-major)   -> columns [256, 384), whole unit
 //   dQ  = dS K       (A = dS from shared memory, M-major; B = K read MN-major) -> columns [0, 128)
 //   dK += dS^T Q     (A = dS^T in TMEM, B = Q read MN-major)   -> columns [384, 512), whole unit
-//   the same warps read dQ out (thread = query row) while dK runs, stage it in the step's Q / dO
-//   buffer, and the TMA unit adds it into an fp32 accumulator (cp.reduce.async.bulk.tensor ... add);
-//   the warps whose boxes go into the Q tile wait for dK, its last reader.
+//   a warpgroup of its own reads dQ out (thread = query row) while dK runs, stages it in the step's
+//   Q / dO buffer, and the TMA unit adds it into an fp32 accumulator (cp.reduce.async.bulk.tensor
+//   ... add); the boxes that go into the Q tile wait for dK, its last reader. Meanwhile the
+//   elementwise warps go on to the next step.
 // MMAs issued by one thread execute in issue order, so dQ may overwrite P^T's columns after the dV
 // product that reads them, and the next step's dP^T may overwrite dS^T's after the dK product; the
 // next step's S^T waits until dQ has been read out of its columns. Eight
@@ -31,6 +32,8 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <atomic>
+
 #include "attn_internal.h"
 #include "sm100_ptx.cuh"
 
@@ -42,13 +45,15 @@ constexpr int BM = 128;                       // query rows per step
 constexpr int BN = 128;                       // keys per CTA
 constexpr int CHUNK_BYTES = 128 * 128;        // 64-column chunk of a 128-row tile (128-byte rows)
 constexpr int TILE_BYTES = 2 * CHUNK_BYTES;   // 128 x 128 bf16
-#ifndef ATTN_BWD_WARPS
-#define ATTN_BWD_WARPS 8
-#endif
-constexpr int NSW = ATTN_BWD_WARPS;           // softmax / epilogue warps: NSW / 4 per TMEM lane quadrant
+constexpr int NSW = 8;                        // softmax / epilogue warps: two per TMEM lane quadrant
 constexpr int CPW = 16 / NSW;                 // 32-column chunks of a 128-column tile per warp
-static_assert(NSW == 8 || NSW == 16, "8 or 16 elementwise warps");
-constexpr int THREADS = 128 + 32 * NSW;
+constexpr int NDQ = 4;                        // dQ warps: one per TMEM lane quadrant
+constexpr int THREADS = 128 + 32 * NSW + 32 * NDQ;
+// register split (setmaxnreg) per warpgroup: control, elementwise (two warpgroups), dQ; the sum must
+// fit in the launch allocation (THREADS x the kernel's register count, checked on the host)
+constexpr int CTRL_REGS = 96;
+constexpr int EW_REGS = 152;
+constexpr int DQ_REGS = 112;
 constexpr int TMEM_COLS = 512;
 constexpr int S_COL = 0, DP_COL = 128, DV_COL = 256, DK_COL = 384;
 // shared memory (tiles first, 1024-byte aligned): K, V, dS, then Q and dO of two stages; then the
@@ -144,12 +149,12 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
     mbar_init(kv_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], NSW);  // the softmax warps release a stage (its space stages dQ last)
+      mbar_init(&q_empty[i], NDQ);  // the dQ warps release a stage (its space stages dQ last)
     }
     mbar_init(s_full, 1);
     mbar_init(p_full, NSW);   // one arrival per softmax warp
     mbar_init(dq_full, 1);
-    mbar_init(dq_free, NSW);  // one arrival per softmax warp
+    mbar_init(dq_free, NDQ);  // one arrival per dQ warp
     mbar_init(dkv_full, 1);
     mbar_init(dk_done, 1);
     *abort_flag = 0;
@@ -171,6 +176,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
 
   if (warp == 0) {
     // ================================ TMA producer ================================
+    regs_dec<CTRL_REGS>();
     if (lane == 0 && n_steps > 0) {
       prefetch_tensormap(&tmQ);
       prefetch_tensormap(&tmK);
@@ -206,6 +212,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ================================ MMA issuer ================================
+    regs_dec<CTRL_REGS>();
     if (lane == 0 && n_steps > 0) {
       // K-major reads of K, V, Q, dO (rows of d) and MN-major reads of Q, dO, K and the dS tile
       const uint64_t dK_k = smem_desc(smem_u32(smem + OFF_K), 16, 1024, kLayoutSW128);
@@ -276,8 +283,86 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
       }
     }
     __syncwarp();
-  } else if (warp >= 4) {
-    // ========================= softmax / dQ / dK dV epilogue warps =========================
+  } else if (warp < 4) {
+    regs_dec<CTRL_REGS>();
+  } else if (warp >= 4 + NSW) {
+    // ================================ dQ warps ================================
+    // Per step, thread = query row q0 + row: once the dQ product is done, read it from TMEM (columns
+    // 64..127 first, staged at once into the step's dO tile, read last by dV, done; then 0..63, after
+    // which the columns are released once dK is done too) and stage it as four 32 x 32 fp32 boxes
+    // (128-byte rows, swizzled like the tensor map): box c of this warp at c * 16 KB + wq * 4 KB, so
+    // boxes 0 and 1 land in the Q tile, which they may overwrite once dK (its last reader) is done. The TMA unit adds the boxes
+    // into the fp32 accumulator; once it has read them the buffer goes back to the producer.
+    regs_dec<DQ_REGS>();
+    const int wq = warp & 3;
+    const uint32_t lane_addr = tmem + (uint32_t(wq * 32) << 16);
+    auto wait_warp = [&](uint64_t* bar, uint32_t ph) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, ph, abort_flag, T));
+    };
+    auto stage_box = [&](uint8_t* box, const uint32_t* o) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t a = smem_u32(box) + lane * 128 + ((u ^ (lane & 7)) << 4);
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(o[4 * u]), "r"(o[4 * u + 1]),
+                     "r"(o[4 * u + 2]), "r"(o[4 * u + 3])
+                     : "memory");
+      }
+    };
+    for (int t = 0; t < n_steps; ++t) {
+      int h, qt;
+      step_coords(t, h, qt);
+      const int row0 = qt * BM + wq * 32;  // first query row of this warp's boxes
+      uint8_t* buf = smem + OFF_Q0 + 2 * (t & 1) * TILE_BYTES + wq * 4096;
+      if (!wait_warp(dq_full, uint32_t(t & 1))) break;
+      tc_fence_after();
+      {
+        uint32_t o[2][32];
+        tmem_ld32(lane_addr + S_COL + 64, o[0]);
+        tmem_ld32(lane_addr + S_COL + 96, o[1]);
+        tmem_ld_wait();
+        tmem_reg_fence32(o[0]);
+        tmem_reg_fence32(o[1]);
+        stage_box(buf + 2 * 16384, o[0]);
+        stage_box(buf + 3 * 16384, o[1]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && row0 < args.Nq) {  // rows past Nq are clipped by the TMA unit
+        tma_reduce_add_4d(&tmDQ, buf + 2 * 16384, 64, h, row0, b);
+        tma_reduce_add_4d(&tmDQ, buf + 3 * 16384, 96, h, row0, b);
+      }
+      uint32_t o[2][32];
+      tmem_ld32(lane_addr + S_COL, o[0]);
+      tmem_ld32(lane_addr + S_COL + 32, o[1]);
+      tmem_ld_wait();
+      tmem_reg_fence32(o[0]);
+      tmem_reg_fence32(o[1]);
+      // dK of this step is done before the columns are released: the next step's dK (whose commit
+      // completes the next phase of dk_done) runs only after the MMAs that wait for the release, so
+      // this wait cannot miss its phase
+      if (!wait_warp(dk_done, uint32_t(t & 1))) break;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_free);
+      stage_box(buf, o[0]);
+      stage_box(buf + 16384, o[1]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (row0 < args.Nq) {
+          tma_reduce_add_4d(&tmDQ, buf, 0, h, row0, b);
+          tma_reduce_add_4d(&tmDQ, buf + 16384, 32, h, row0, b);
+        }
+        bulk_commit_group();
+        bulk_wait_group_read0();  // the TMA unit has read the boxes: the buffer may be refilled
+        mbar_arrive(&q_empty[t & 1]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) bulk_wait_group0();  // this warp's dQ additions have been performed
+  } else {
+    // ========================= softmax / dK dV epilogue warps =========================
+    regs_inc<EW_REGS>();
     const int wq = warp & 3;
     const int cw = (warp - 4) >> 2;   // which CPW x 32 of the 128 columns this warp covers
     const int row = wq * 32 + lane;   // TMEM lane: key row (softmax, dK dV) or query row (dQ)
@@ -360,59 +445,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
-      // the previous step's dQ boxes (in that step's Q / dO buffer) have been read by the TMA unit
-      // by now, as a rule: hand the buffer back to the producer for the step after this one
-      if (t > 0 && lane == 0) {
-        bulk_wait_group_read0();
-        mbar_arrive(&q_empty[(t - 1) & 1]);
-      }
-      // dQ of this step (thread = query row q0 + row, this warp's 64 of the d columns): once the dQ
-      // product is done, read it from TMEM and release those columns, then stage it as two 32 x 32
-      // fp32 boxes (128-byte rows, swizzled like the tensor map) in this step's Q / dO buffer, and
-      // let the TMA unit add the boxes into the fp32 accumulator. The buffer goes back to the
-      // producer once the TMA has read it (checked one step later, above).
-      if (!wait_warp(dq_full, uint32_t(t & 1))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t o[CPW][32];
-#pragma unroll
-      for (int cx = 0; cx < CPW; ++cx) tmem_ld32(lane_addr + S_COL + (CPW * cw + cx) * 32, o[cx]);
-      tmem_ld_wait();
-#pragma unroll
-      for (int cx = 0; cx < CPW; ++cx) tmem_reg_fence32(o[cx]);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dq_free);
-      const int row0 = q0 + wq * 32;  // first query row of this warp's boxes
-      // the second half of the warps stage into the step's dO tile, read last by dV (done); the first
-      // half into its Q tile, read last by dK, which runs after dQ: those wait for it
-      const int box_off = (warp - 4) * CPW * 4096;
-      if (box_off < TILE_BYTES && !wait_warp(dk_done, uint32_t(t & 1))) {
-        ok = false;
-        break;
-      }
-      uint8_t* box = smem + OFF_Q0 + 2 * (t & 1) * TILE_BYTES + box_off;
-#pragma unroll
-      for (int cx = 0; cx < CPW; ++cx)
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const uint32_t a = smem_u32(box + cx * 4096) + lane * 128 + ((u ^ (lane & 7)) << 4);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(o[cx][4 * u]), "r"(o[cx][4 * u + 1]),
-                       "r"(o[cx][4 * u + 2]), "r"(o[cx][4 * u + 3])
-                       : "memory");
-        }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0 && row0 < args.Nq) {  // rows past Nq are clipped by the TMA unit
-#pragma unroll
-        for (int cx = 0; cx < CPW; ++cx) tma_reduce_add_4d(&tmDQ, box + cx * 4096, (CPW * cw + cx) * 32, h, row0, b);
-        bulk_commit_group();
-      }
-      __syncwarp();
     }
-    if (lane == 0) bulk_wait_group0();  // this warp's dQ additions have been performed
     // dK (times scale) and dV of this key block, bf16, this warp's 64 of the d columns
     if (key_ok && n_steps == 0) {
       for (int which = 0; which < 2; ++which) {
@@ -526,6 +559,20 @@ attn_status_t bwd_dispatch(const void* q, const void* k, const void* v, const vo
     if (!encode_map(&tmDQ, acc, 4, dims, box, 128)) return ATTN_ERR_CUDA;
   }
   if (ensure_dyn_smem(reinterpret_cast<const void*>(attn_bwd_kernel), SMEM_BYTES) != cudaSuccess) return ATTN_ERR_CUDA;
+  {
+    // setmaxnreg.inc waits until the registers it asks for are free in the CTA's launch allocation,
+    // so a split whose total exceeds that allocation would never proceed: refuse to launch it
+    static std::atomic<int> regs_ok{0};  // 0 unknown, 1 fits, 2 does not (same binary on every device)
+    int st = regs_ok.load(std::memory_order_relaxed);
+    if (st == 0) {
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, attn_bwd_kernel) != cudaSuccess) return ATTN_ERR_CUDA;
+      const long long need = 128LL * (CTRL_REGS + 2 * EW_REGS + DQ_REGS);
+      st = (long long)fa.numRegs * THREADS >= need ? 1 : 2;
+      regs_ok.store(st, std::memory_order_relaxed);
+    }
+    if (st != 1) return ATTN_ERR_UNSUPPORTED;
+  }
   if (cudaMemsetAsync(acc, 0, acc_bytes, stream) != cudaSuccess) return ATTN_ERR_CUDA;
   attn_bwd_pre_kernel<<<dim3(Nq_pad / 128, B * Hq), 128, 0, stream>>>(
       reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dout), lse, lse2, dd, Nq, Hq,
