@@ -300,7 +300,6 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
   if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID_ARG;
   if (d != 128) return ATTN_ERR_UNSUPPORTED;
-  if ((long long)B * Hq > 65535) return ATTN_ERR_UNSUPPORTED;  // grid y of the row passes
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
       workspace_bytes < bwd_workspace(B, Hq, Nq, d))
     return ATTN_ERR_WORKSPACE;

@@ -65,8 +65,8 @@ constexpr int OFF_K = 0, OFF_V = TILE_BYTES, OFF_DS = 2 * TILE_BYTES;
 constexpr int OFF_Q0 = 3 * TILE_BYTES;        // stage s: Q at OFF_Q0 + 2s tiles, dO right after it
 constexpr int OFF_LSE0 = 7 * TILE_BYTES;      // stage s: LSE' at OFF_LSE0 + s * 1024, D 512 bytes later
 constexpr int OFF_BAR = OFF_LSE0 + 2 * 1024;
-// kv_full, q_full[2], q_empty[2], s_full, p_full, dq_full, dq_free, dkv_full, dk_done
-constexpr int NBARS = 11;
+// kv_full, q_full[2], q_empty[2], s_full, p_full, dq_full, dq_free, dkv_full, dk_done, epi_full, epi_free
+constexpr int NBARS = 13;
 constexpr int SMEM_BYTES = OFF_BAR + NBARS * 8 + 16;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 }  // namespace bwd
@@ -102,6 +102,16 @@ __device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const 
       : "memory");
 }
 
+// Stores a shared-memory box to global memory through the TMA unit (rows and columns outside the
+// tensor are not written), tracked by the issuing thread's bulk async-group.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* smem_src, int c0, int c1, int c2,
+                                             int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+
 // First query tile whose rows see some key of block kb (causal: key j visible to row i iff
 // j <= i + Nkv - Nq).
 __device__ __forceinline__ int first_q_tile(const BwdArgs& a, int kb) {
@@ -113,7 +123,8 @@ __device__ __forceinline__ int first_q_tile(const BwdArgs& a, int kb) {
 __global__ void __launch_bounds__(bwd::THREADS, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const __grid_constant__ CUtensorMap tmDQ, const BwdArgs args) {
+                    const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmDK,
+                    const __grid_constant__ CUtensorMap tmDV, const BwdArgs args) {
   using namespace bwd;
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_u32(smem) & 1023u) != 0) {
@@ -130,6 +141,8 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
   uint64_t* dq_free = bars + 8;
   uint64_t* dkv_full = bars + 9;
   uint64_t* dk_done = bars + 10;  // one phase per step: the step's dK product (the last reader of Q) is done
+  uint64_t* epi_full = bars + 11; // one phase per dK / dV tile: staged in shared memory by every warp
+  uint64_t* epi_free = bars + 12; // one phase per dK / dV tile: the TMA unit has read it
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -157,6 +170,8 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
     mbar_init(dq_free, NDQ);  // one arrival per dQ warp
     mbar_init(dkv_full, 1);
     mbar_init(dk_done, 1);
+    mbar_init(epi_full, NSW);  // one arrival per elementwise warp
+    mbar_init(epi_free, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -359,7 +374,12 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
       }
       __syncwarp();
     }
-    if (lane == 0) bulk_wait_group0();  // this warp's dQ additions have been performed
+    // The additions still in flight complete with the kernel; the CTA may exit once the TMA unit has
+    // read their shared-memory sources (done after every step; here for a step left by an error).
+    if (lane == 0) {
+      bulk_commit_group();
+      bulk_wait_group_read0();
+    }
   } else {
     // ========================= softmax / dK dV epilogue warps =========================
     regs_inc<EW_REGS>();
@@ -456,28 +476,46 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
     }
     if (n_steps > 0 && ok && wait_warp(dkv_full, 0)) {
       tc_fence_after();
+      // Staged in the dS tile (free: every MMA is done), 128-byte swizzled like the tensor maps
+      // (this warp's 64 columns are box cw), and written by TMA stores, dK first; the tile is
+      // reused for dV once the TMA unit has read it.
 #pragma unroll 1
       for (int which = 0; which < 2; ++which) {
         const float mul = which == 0 ? args.scale : 1.0f;
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(which == 0 ? args.dk : args.dv) +
-                             ((size_t(b) * args.Nkv + (key_ok ? key : 0)) * args.Hkv + g) * D;
 #pragma unroll 1
         for (int cx = 0; cx < CPW; ++cx) {
-          const int cc = CPW * cw + cx;
           uint32_t o[32];
-          tmem_ld32(lane_addr + (which == 0 ? DK_COL : DV_COL) + cc * 32, o);
+          tmem_ld32(lane_addr + (which == 0 ? DK_COL : DV_COL) + (CPW * cw + cx) * 32, o);
           tmem_ld_wait();
           tmem_reg_fence32(o);
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * mul, __uint_as_float(o[2 * i + 1]) * mul);
-          if (key_ok) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4) d4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          for (int v4 = 0; v4 < 4; ++v4) {
+            const int unit = cx * 4 + v4;  // 16-byte unit of the row's 128 bytes
+            const uint32_t addr = smem_u32(smem + OFF_DS) + cw * CHUNK_BYTES + row * 128 + ((unit ^ (row & 7)) << 4);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * v4]), "r"(pk[4 * v4 + 1]),
+                         "r"(pk[4 * v4 + 2]), "r"(pk[4 * v4 + 3])
+                         : "memory");
           }
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(epi_full);
+        if (warp == 4 && lane == 0) {
+          // every warp's rows are in: store the tile, and free it once the TMA unit has read it
+          if (mbar_wait(epi_full, uint32_t(which), abort_flag, T)) {
+            const CUtensorMap* m = which == 0 ? &tmDK : &tmDV;
+            tma_store_4d(m, smem + OFF_DS, 0, g, kb * BN, b);
+            tma_store_4d(m, smem + OFF_DS + CHUNK_BYTES, 64, g, kb * BN, b);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+            mbar_arrive(epi_free);
+          }
+        }
+        if (!wait_warp(epi_free, uint32_t(which))) break;
       }
     }
   }
@@ -490,34 +528,56 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
   }
 }
 
-// D_i = sum_e dO_ie O_ie and LSE'_i = LSE_i * log2 e (+inf when the row has no key), per (b, h) row of
-// whole tiles (padding rows: +inf and 0).
-__global__ void __launch_bounds__(128)
+// D_i = sum_e dO_ie O_ie and LSE'_i = LSE_i * log2 e (+inf when the row has no key) per (b, i, h) row,
+// and the row of the fp32 dQ accumulator zeroed. Rows are taken in memory order, 16 lanes per row
+// (16 bytes of O, of dO and 32 bytes of the accumulator each), so every access is coalesced; the
+// 16-lane partial sums are combined by shuffles. The padding entries of the LSE' / D rows (whole
+// tiles) get +inf and 0.
+__global__ void __launch_bounds__(256)
     attn_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
-                        const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ dd, int Nq,
-                        int Hq, int Nq_pad) {
-  const int bh = blockIdx.y, b = bh / Hq, h = bh % Hq;
-  const int i = blockIdx.x * 128 + threadIdx.x;
-  if (i >= Nq_pad) return;
-  float l2 = INFINITY, dsum = 0.f;
-  if (i < Nq) {
-    const float L = lse[size_t(bh) * Nq + i];
-    l2 = (L == -INFINITY) ? INFINITY : L * 1.4426950408889634f;
-    const uint4* po = reinterpret_cast<const uint4*>(o + ((size_t(b) * Nq + i) * Hq + h) * bwd::D);
-    const uint4* pd = reinterpret_cast<const uint4*>(dout + ((size_t(b) * Nq + i) * Hq + h) * bwd::D);
-#pragma unroll 4
-    for (int u = 0; u < bwd::D / 8; ++u) {
-      const uint4 a = po[u], c = pd[u];
+                        const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ dd,
+                        float* __restrict__ acc, int B, int Nq, int Hq, int Nq_pad) {
+  const long long rows = (long long)B * Nq * Hq;
+  const int lane = threadIdx.x & 31, seg = lane & 15;
+  const long long warp_g = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
+  const long long n_warps = (gridDim.x * (long long)blockDim.x) >> 5;
+  for (long long r = 2 * warp_g + (lane >> 4); r - (lane >> 4) < rows; r += 2 * n_warps) {
+    const bool valid = r < rows;
+    float dsum = 0.f;
+    if (valid) {
+      const uint4 a = reinterpret_cast<const uint4*>(o + r * bwd::D)[seg];
+      const uint4 c = reinterpret_cast<const uint4*>(dout + r * bwd::D)[seg];
       const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wc[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         dsum = fmaf(__uint_as_float(wa[k] << 16), __uint_as_float(wc[k] << 16), dsum);
         dsum = fmaf(__uint_as_float(wa[k] & 0xFFFF0000u), __uint_as_float(wc[k] & 0xFFFF0000u), dsum);
       }
+      float4* z = reinterpret_cast<float4*>(acc + r * bwd::D) + 2 * seg;
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
+    if (valid && seg == 0) {
+      const int h = int(r % Hq);
+      const long long bi = r / Hq;
+      const int i = int(bi % Nq), b = int(bi / Nq);
+      const size_t bh = size_t(b) * Hq + h;
+      const float L = lse[bh * Nq + i];
+      lse2[bh * Nq_pad + i] = (L == -INFINITY) ? INFINITY : L * 1.4426950408889634f;
+      dd[bh * Nq_pad + i] = dsum;
     }
   }
-  lse2[size_t(bh) * Nq_pad + i] = l2;
-  dd[size_t(bh) * Nq_pad + i] = dsum;
+  // padding entries i in [Nq, Nq_pad) of every (b, h) row
+  const int pad = Nq_pad - Nq;
+  const long long n_pad = (long long)B * Hq * pad;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n_pad; e += gridDim.x * (long long)blockDim.x) {
+    const long long bh = e / pad;
+    const int i = Nq + int(e % pad);
+    lse2[bh * Nq_pad + i] = INFINITY;
+    dd[bh * Nq_pad + i] = 0.f;
+  }
 }
 
 // dQ = scale * accumulator, bf16
@@ -552,6 +612,10 @@ attn_status_t bwd_dispatch(const void* q, const void* k, const void* v, const vo
       !encode_tile_map(&tmV, v, D, Hkv, Nkv, B, 64, BN, 128) ||
       !encode_tile_map(&tmDO, dout, D, Hq, Nq, B, 64, BM, 128))
     return ATTN_ERR_CUDA;
+  // dK and dV are written by TMA stores of 64-column boxes of a key block
+  CUtensorMap tmDK, tmDV;
+  if (!encode_tile_map(&tmDK, dk, D, Hkv, Nkv, B, 64, BN, 128) || !encode_tile_map(&tmDV, dv, D, Hkv, Nkv, B, 64, BN, 128))
+    return ATTN_ERR_CUDA;
   CUtensorMap tmDQ;
   {
     const long long dims[4] = {D, Hq, Nq, B};
@@ -573,10 +637,17 @@ attn_status_t bwd_dispatch(const void* q, const void* k, const void* v, const vo
     }
     if (st != 1) return ATTN_ERR_UNSUPPORTED;
   }
-  if (cudaMemsetAsync(acc, 0, acc_bytes, stream) != cudaSuccess) return ATTN_ERR_CUDA;
-  attn_bwd_pre_kernel<<<dim3(Nq_pad / 128, B * Hq), 128, 0, stream>>>(
-      reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dout), lse, lse2, dd, Nq, Hq,
-      Nq_pad);
+  {
+    // the row pass: rows are 16-lane groups, two per warp; about 16 warps per SM in flight
+    const long long rows = (long long)B * Nq * Hq;
+    const int n_sm = sm_count();
+    if (n_sm <= 0) return ATTN_ERR_CUDA;
+    const long long want = (rows + 15) / 16;  // blocks of 8 warps, 16 rows per block and iteration
+    const long long cap = (long long)n_sm * 8;
+    attn_bwd_pre_kernel<<<dim3(unsigned(want < cap ? want : cap)), 256, 0, stream>>>(
+        reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dout), lse, lse2, dd, acc, B,
+        Nq, Hq, Nq_pad);
+  }
   BwdArgs a;
   a.dk = dk;
   a.dv = dv;
@@ -597,7 +668,7 @@ attn_status_t bwd_dispatch(const void* q, const void* k, const void* v, const vo
   a.timeout_ns = kWaitLimitNs;
   const long long grid = (long long)a.n_kb * B * Hkv;
   if (grid > 0x7FFFFFFFll) return ATTN_ERR_UNSUPPORTED;
-  attn_bwd_kernel<<<dim3(unsigned(grid)), THREADS, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmDO, tmDQ, a);
+  attn_bwd_kernel<<<dim3(unsigned(grid)), THREADS, SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmDO, tmDQ, tmDK, tmDV, a);
   const size_t n4 = size_t(B) * Nq * Hq * D / 4;
   attn_bwd_post_kernel<<<dim3(unsigned(n4 / 256 + 1 < 8192 ? n4 / 256 + 1 : 8192)), 256, 0, stream>>>(
       acc, reinterpret_cast<__nv_bfloat16*>(dq), n4, scale);

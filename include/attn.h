@@ -119,7 +119,7 @@ attn_status_t attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, cons
  *   dq          bf16 [B, Nq, Hq, d];  dk, dv bf16 [B, Nkv, Hkv, d], written
  *   workspace   caller-owned, at least attn_bwd_workspace_bytes(B, Hq, Nq, d) bytes, 256-byte
  *               aligned, no initialisation needed (the call zeroes what it accumulates into)
- *   d = 128 (ATTN_ERR_UNSUPPORTED otherwise); B * Hq <= 65535; everything else as attn_fwd.
+ *   d = 128 (ATTN_ERR_UNSUPPORTED otherwise); everything else as attn_fwd.
  */
 size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq, int d);
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,

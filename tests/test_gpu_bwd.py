@@ -74,6 +74,15 @@ def test_backward_gqa_and_large_scale(lib):
     _run(lib, 8101, 1, 4, 1, 256, 320, False, scale=0.5)
 
 
+def test_backward_more_units_than_sms(lib):
+    # 6 key blocks x 4 batches x 8 kv heads = 192 key-block CTAs, more than one wave on 148 SMs, with
+    # causal units of 1 to 6 steps, key blocks that end ragged (700 keys), a non-causal GQA case, and
+    # 100 queries against 700 keys (causal: one step per key block)
+    _run(lib, 8200, 4, 8, 8, 700, 700, True)
+    _run(lib, 8201, 4, 16, 8, 700, 700, False)
+    _run(lib, 8202, 4, 8, 8, 100, 700, True)
+
+
 def test_backward_causal_2k_workload_whole_tensors(lib):
     import torch
 
