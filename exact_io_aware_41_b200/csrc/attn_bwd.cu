@@ -65,8 +65,8 @@ constexpr int OFF_K = 0, OFF_V = TILE_BYTES, OFF_DS = 2 * TILE_BYTES;
 constexpr int OFF_Q0 = 3 * TILE_BYTES;        // stage s: Q at OFF_Q0 + 2s tiles, dO right after it
 constexpr int OFF_LSE0 = 7 * TILE_BYTES;      // stage s: LSE' at OFF_LSE0 + s * 1024, D 512 bytes later
 constexpr int OFF_BAR = OFF_LSE0 + 2 * 1024;
-// kv_full, q_full[2], q_empty[2], s_full, p_full, dq_full, dq_free, dkv_full, dk_done, epi_full, epi_free
-constexpr int NBARS = 13;
+// kv_full, q_full[2], q_empty[2], s_full, p_full, dq_full, dq_free, dkv_full, dk_done[2], epi_full, epi_free
+constexpr int NBARS = 14;
 constexpr int SMEM_BYTES = OFF_BAR + NBARS * 8 + 16;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 }  // namespace bwd
@@ -140,9 +140,10 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
   uint64_t* dq_full = bars + 7;
   uint64_t* dq_free = bars + 8;
   uint64_t* dkv_full = bars + 9;
-  uint64_t* dk_done = bars + 10;  // one phase per step: the step's dK product (the last reader of Q) is done
-  uint64_t* epi_full = bars + 11; // one phase per dK / dV tile: staged in shared memory by every warp
-  uint64_t* epi_free = bars + 12; // one phase per dK / dV tile: the TMA unit has read it
+  uint64_t* dk_done = bars + 10;  // [2] step t's dK product (the last reader of its Q tile) is done: slot
+                                  // t & 1, one phase per two steps
+  uint64_t* epi_full = bars + 12; // one phase per dK / dV tile: staged in shared memory by every warp
+  uint64_t* epi_free = bars + 13; // one phase per dK / dV tile: the TMA unit has read it
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -169,7 +170,8 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
     mbar_init(dq_full, 1);
     mbar_init(dq_free, NDQ);  // one arrival per dQ warp
     mbar_init(dkv_full, 1);
-    mbar_init(dk_done, 1);
+    mbar_init(&dk_done[0], 1);
+    mbar_init(&dk_done[1], 1);
     mbar_init(epi_full, NSW);  // one arrival per elementwise warp
     mbar_init(epi_free, 1);
     *abort_flag = 0;
@@ -287,7 +289,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
         for (int kk = 0; kk < BM / 16; ++kk)
           umma_ts(tmem + DK_COL, tmem + DP_COL + 32 * (kk / 2) + 8 * (kk % 2),
                   dQ_mn + uint64_t((kk * 16 * 128) >> 4), idesc_tmn, (t > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(dk_done);
+        umma_commit(&dk_done[t & 1]);
         if (t == n_steps - 1) umma_commit(dkv_full);
       }
       if (!ok) {
@@ -352,13 +354,13 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
       tmem_ld_wait();
       tmem_reg_fence32(o[0]);
       tmem_reg_fence32(o[1]);
-      // dK of this step is done before the columns are released: the next step's dK (whose commit
-      // completes the next phase of dk_done) runs only after the MMAs that wait for the release, so
-      // this wait cannot miss its phase
-      if (!wait_warp(dk_done, uint32_t(t & 1))) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_free);
+      // the Q tile may take the boxes once dK (its last reader) is done. Step t's dK completes slot
+      // t & 1; the slot's next phase needs step t + 2's dK, which runs only after this warp has
+      // released step t + 1's columns, so this wait cannot miss its phase
+      if (!wait_warp(&dk_done[t & 1], uint32_t((t >> 1) & 1))) break;
       stage_box(buf, o[0]);
       stage_box(buf + 16384, o[1]);
       fence_proxy_async_smem();
