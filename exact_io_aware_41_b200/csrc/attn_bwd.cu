@@ -52,8 +52,8 @@ constexpr int THREADS = 128 + 32 * NSW + 32 * NDQ;
 // register split (setmaxnreg) per warpgroup: control, elementwise (two warpgroups), dQ; the sum must
 // fit in the launch allocation (THREADS x the kernel's register count, checked on the host)
 constexpr int CTRL_REGS = 96;
-constexpr int EW_REGS = 152;
-constexpr int DQ_REGS = 112;
+constexpr int EW_REGS = 160;
+constexpr int DQ_REGS = 96;
 constexpr int TMEM_COLS = 512;
 constexpr int S_COL = 0, DP_COL = 128, DV_COL = 256, DK_COL = 384;
 // shared memory (tiles first, 1024-byte aligned): K, V, dS, then Q and dO of two stages; then the
@@ -65,8 +65,9 @@ constexpr int OFF_K = 0, OFF_V = TILE_BYTES, OFF_DS = 2 * TILE_BYTES;
 constexpr int OFF_Q0 = 3 * TILE_BYTES;        // stage s: Q at OFF_Q0 + 2s tiles, dO right after it
 constexpr int OFF_LSE0 = 7 * TILE_BYTES;      // stage s: LSE' at OFF_LSE0 + s * 1024, D 512 bytes later
 constexpr int OFF_BAR = OFF_LSE0 + 2 * 1024;
-// kv_full, q_full[2], q_empty[2], s_full, p_full, dq_full, dq_free, dkv_full, dk_done[2], epi_full, epi_free
-constexpr int NBARS = 14;
+// kv_full, q_full[2], q_empty[2], s_full, p_full, dq_full, dq_free, dkv_full, dk_done[2], epi_full, epi_free,
+// st_full
+constexpr int NBARS = 15;
 constexpr int SMEM_BYTES = OFF_BAR + NBARS * 8 + 16;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 }  // namespace bwd
@@ -144,6 +145,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
                                   // t & 1, one phase per two steps
   uint64_t* epi_full = bars + 12; // one phase per dK / dV tile: staged in shared memory by every warp
   uint64_t* epi_free = bars + 13; // one phase per dK / dV tile: the TMA unit has read it
+  uint64_t* st_full = bars + 14;  // one phase per step: S^T is in (s_full: dP^T too)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -166,6 +168,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
       mbar_init(&q_empty[i], NDQ);  // the dQ warps release a stage (its space stages dQ last)
     }
     mbar_init(s_full, 1);
+    mbar_init(st_full, 1);
     mbar_init(p_full, NSW);   // one arrival per softmax warp
     mbar_init(dq_full, 1);
     mbar_init(dq_free, NDQ);  // one arrival per dQ warp
@@ -261,6 +264,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
           const uint32_t off = ((kk / 4) * CHUNK_BYTES + (kk % 4) * 32) >> 4;
           umma_ss(tmem + S_COL, dK_k + off, dQ_k + off, idesc_kk, kk > 0 ? 1u : 0u);
         }
+        umma_commit(st_full);  // the elementwise warps start on P while dP^T runs
         // dP^T = V dO^T into [128, 256): dS^T of the previous step there was read by its dK product,
         // issued earlier by this thread
 #pragma unroll
@@ -402,31 +406,30 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
       step_coords(t, h, qt);
       const float* s_lse = reinterpret_cast<const float*>(smem + OFF_LSE0 + (t & 1) * 1024);
       const float* s_dd = s_lse + 128;
-      if (!wait_warp(s_full, uint32_t(t & 1))) {
+      const int q0 = qt * BM;
+      // P first, from S^T alone (its product is done before dP^T's), kept in fp32 for dS
+      if (!wait_warp(st_full, uint32_t(t & 1))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int q0 = qt * BM;
-#pragma unroll 1
+      float pf[CPW][32];
+#pragma unroll
       for (int cx = 0; cx < CPW; ++cx) {  // 32 query columns at a time, this warp's CPW x 32
         const int cc = CPW * cw + cx;
-        uint32_t sv[32], dpv[32];
+        uint32_t sv[32];
         tmem_ld32(lane_addr + S_COL + cc * 32, sv);
-        tmem_ld32(lane_addr + DP_COL + cc * 32, dpv);
         tmem_ld_wait();
         tmem_reg_fence32(sv);
-        tmem_reg_fence32(dpv);
         // warp-uniform: does some (key, query) of this 32 x 32 block fall outside the mask? (rows
         // past Nq need no test: their LSE' is +inf, so P = 0)
         const int qf = q0 + cc * 32;
         const bool need_mask = (kb * BN + BN > args.Nkv) || (args.causal && kb * BN + BN - 1 > qf + diag);
-        uint32_t pk[16], dk2[16];
+        uint32_t pk[16];
 #pragma unroll
         for (int i4 = 0; i4 < 8; ++i4) {
           const float4 l4 = *reinterpret_cast<const float4*>(s_lse + cc * 32 + 4 * i4);
-          const float4 d4 = *reinterpret_cast<const float4*>(s_dd + cc * 32 + 4 * i4);
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
           // pairs of query columns on the packed FMA pipe (the same roundings as the scalar forms)
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
@@ -438,16 +441,43 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
               if (!(key_ok && (!args.causal || key <= q0 + qi + diag))) p.x = 0.f;
               if (!(key_ok && (!args.causal || key <= q0 + qi + 1 + diag))) p.y = 0.f;
             }
-            const float2 ds = fmul2(p, fadd2(make_float2(__uint_as_float(dpv[4 * i4 + u]),
-                                                         __uint_as_float(dpv[4 * i4 + u + 1])),
-                                             make_float2(-dv4[u], -dv4[u + 1])));
+            pf[cx][4 * i4 + u] = p.x;
+            pf[cx][4 * i4 + u + 1] = p.y;
             pk[2 * i4 + h2] = pack_bf16x2(p.x, p.y);
+          }
+        }
+        // P^T over S^T, bf16 pairs: the chunk's 16 columns go to the first 16 of its own 32 score
+        // columns (just read), so no warp writes where the other still reads
+        tmem_st16(lane_addr + S_COL + cc * 32, pk);
+      }
+      // then dS = P (dP - D), once dP^T is in
+      if (!wait_warp(s_full, uint32_t(t & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int cx = 0; cx < CPW; ++cx) {
+        const int cc = CPW * cw + cx;
+        uint32_t dpv[32];
+        tmem_ld32(lane_addr + DP_COL + cc * 32, dpv);
+        tmem_ld_wait();
+        tmem_reg_fence32(dpv);
+        uint32_t dk2[16];
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 d4 = *reinterpret_cast<const float4*>(s_dd + cc * 32 + 4 * i4);
+          const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int u = 2 * h2;
+            const float2 ds = fmul2(make_float2(pf[cx][4 * i4 + u], pf[cx][4 * i4 + u + 1]),
+                                    fadd2(make_float2(__uint_as_float(dpv[4 * i4 + u]), __uint_as_float(dpv[4 * i4 + u + 1])),
+                                          make_float2(-dv4[u], -dv4[u + 1])));
             dk2[2 * i4 + h2] = pack_bf16x2(ds.x, ds.y);
           }
         }
-        // P^T over S^T and dS^T over dP^T, bf16 pairs: the chunk's 16 columns go to the first 16 of
-        // its own 32 score columns (just read), so no warp writes where the other still reads
-        tmem_st16(lane_addr + S_COL + cc * 32, pk);
+        // dS^T over dP^T, as P^T over S^T
         tmem_st16(lane_addr + DP_COL + cc * 32, dk2);
         // dS^T row into the shared tile [key][query] (128-byte swizzled, 64-query chunks): the A
         // operand of dQ = dS K, read M-major
