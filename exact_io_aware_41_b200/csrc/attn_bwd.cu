@@ -66,8 +66,8 @@ constexpr int OFF_Q0 = 3 * TILE_BYTES;        // stage s: Q at OFF_Q0 + 2s tiles
 constexpr int OFF_LSE0 = 7 * TILE_BYTES;      // stage s: LSE' at OFF_LSE0 + s * 1024, D 512 bytes later
 constexpr int OFF_BAR = OFF_LSE0 + 2 * 1024;
 // kv_full, q_full[2], q_empty[2], s_full, p_full, dq_full, dq_free, dkv_full, dk_done[2], epi_full, epi_free,
-// st_full
-constexpr int NBARS = 15;
+// st_full, pt_full
+constexpr int NBARS = 16;
 constexpr int SMEM_BYTES = OFF_BAR + NBARS * 8 + 16;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 }  // namespace bwd
@@ -146,6 +146,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
   uint64_t* epi_full = bars + 12; // one phase per dK / dV tile: staged in shared memory by every warp
   uint64_t* epi_free = bars + 13; // one phase per dK / dV tile: the TMA unit has read it
   uint64_t* st_full = bars + 14;  // one phase per step: S^T is in (s_full: dP^T too)
+  uint64_t* pt_full = bars + 15;  // one phase per step: P^T is in (p_full: dS^T too)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -169,6 +170,7 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(st_full, 1);
+    mbar_init(pt_full, NSW);  // one arrival per elementwise warp
     mbar_init(p_full, NSW);   // one arrival per softmax warp
     mbar_init(dq_full, 1);
     mbar_init(dq_free, NDQ);  // one arrival per dQ warp
@@ -273,17 +275,21 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
           umma_ss(tmem + DP_COL, dV_k + off, dDO_k + off, idesc_kk, kk > 0 ? 1u : 0u);
         }
         umma_commit(s_full);
-        ok = mbar_wait(p_full, uint32_t(t & 1), abort_flag, T);
-        if (!ok) break;
-        tc_fence_after();
-        // over the step's 128 queries (k-steps of 16): dV += P^T dO, then dQ = dS K into [0, 128)
-        // (after the dV product has read P^T there), whose read-out overlaps dK += dS^T Q
+        // over the step's 128 queries (k-steps of 16): dV += P^T dO as soon as P^T is in (it runs
+        // while the elementwise warps form dS), then dQ = dS K into [0, 128) (after the dV product
+        // has read P^T there), whose read-out overlaps dK += dS^T Q.
         // A = P^T / dS^T: queries 16kk .. 16kk+15 are columns 8 (kk % 2) .. of chunk kk / 2, which
         // starts at column 32 (kk / 2)
+        ok = mbar_wait(pt_full, uint32_t(t & 1), abort_flag, T);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
           umma_ts(tmem + DV_COL, tmem + S_COL + 32 * (kk / 2) + 8 * (kk % 2),
                   dDO_mn + uint64_t((kk * 16 * 128) >> 4), idesc_tmn, (t > 0 || kk > 0) ? 1u : 0u);
+        ok = mbar_wait(p_full, uint32_t(t & 1), abort_flag, T);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
           umma_ss(tmem + S_COL, dDS_mn + uint64_t((kk * 16 * 128) >> 4), dK_mn + uint64_t((kk * 16 * 128) >> 4),
@@ -450,6 +456,11 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
         // columns (just read), so no warp writes where the other still reads
         tmem_st16(lane_addr + S_COL + cc * 32, pk);
       }
+      // P^T is in tensor memory: the dV product may start
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pt_full);
       // then dS = P (dP - D), once dP^T is in
       if (!wait_warp(s_full, uint32_t(t & 1))) {
         ok = false;
