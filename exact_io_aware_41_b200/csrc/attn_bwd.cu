@@ -9,10 +9,12 @@
 // that sees some of its keys. Per step (all products on tcgen05, accumulators in TMEM):
 //   S^T = K Q^T      (M = keys, N = queries)           -> TMEM columns [0, 128)
 //   dP^T = V dO^T                                      -> TMEM columns [128, 256)
-//   softmax warps (thread = key row): P^T = exp2(S^T * scale * log2 e - LSE * log2 e), masked;
-//   dS^T = P^T * (dP^T - D); P^T (bf16) over S^T, dS^T (bf16) over dP^T (each 32-query chunk's
-//   16 packed columns at the start of its own 32 score columns) and dS^T into shared memory
-//   dV += P^T dO     (A = P^T in TMEM, B = dO read MN-major)   -> columns [256, 384), whole unit
+//   elementwise warps (thread = key row): once S^T is in, P^T = exp2(S^T * scale * log2 e -
+//   LSE * log2 e), masked, P^T (bf16) over S^T (each 32-query chunk's 16 packed columns at the start
+//   of its own 32 score columns); once dP^T is in, dS^T = P^T * (dP^T - D), dS^T (bf16) over dP^T
+//   and dS^T into shared memory
+//   dV += P^T dO     (A = P^T in TMEM, B = dO read MN-major)   -> columns [256, 384), whole unit;
+//                    issued as soon as P^T is in, so it runs while dS is formed
 //   dQ  = dS K       (A = dS from shared memory, M-major; B = K read MN-major) -> columns [0, 128)
 //   dK += dS^T Q     (A = dS^T in TMEM, B = Q read MN-major)   -> columns [384, 512), whole unit
 //   a warpgroup of its own reads dQ out (thread = query row) while dK runs, stages it in the step's
@@ -21,10 +23,11 @@
 //   elementwise warps go on to the next step.
 // MMAs issued by one thread execute in issue order, so dQ may overwrite P^T's columns after the dV
 // product that reads them, and the next step's dP^T may overwrite dS^T's after the dK product; the
-// next step's S^T waits until dQ has been read out of its columns. Eight
-// warps (two per TMEM lane quadrant, 64 of the 128 columns each) do the elementwise work; Q, dO and
-// their LSE' and D rows are double-buffered so the next step's loads overlap this one. The unit ends
-// with dK (times scale) and dV stored as bf16.
+// next step's S^T waits until dQ has been read out of its columns. Eight elementwise warps (two per
+// TMEM lane quadrant, 64 of the 128 columns each) and four dQ warps (one per quadrant), next to the
+// producer and MMA warps; Q, dO and their LSE' and D rows are double-buffered so the next step's
+// loads overlap this one. The unit ends with dK (times scale) and dV converted to bf16 in the dS
+// tile and written by TMA stores.
 //
 // A pre-pass writes D and LSE * log2 e per query row (padded to whole tiles; rows without keys or
 // past Nq get LSE' = +inf, so their P is 0) and zeroes the dQ accumulator; a post-pass rounds
