@@ -39,6 +39,7 @@ METRIC = "attn fwd TFLOP/s & % of BF16 peak (prefill); decode HBM GB/s & % of pe
 NOMINAL_BF16_TFLOPS = 2250.0
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+LONG_REGION_MS = 1000.0  # a timed region at least this long is measured against the sustained peak
 
 
 # DRAM traffic per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum; summaries and commands
@@ -377,7 +378,12 @@ def run_ours(args, world, rank, local, dist):
         dv, dsample, _ = cpu_decode(Dw, args.cpu_budget / 2)
         cpu["decode"] = {"value": dv, "unit": "GB/s", "sample": dsample}
 
-    meas_tf = peaks.get("bf16_tflops", FALLBACK["bf16_tflops"])
+    # the headline kernel is timed inside the step loop: over a seconds-long timed region the GPU
+    # settles at its power-capped clock, so the denominator is the sustained GEMM figure; over a
+    # short one (a few tens of steps) it is the burst figure
+    long_region = total_ms >= LONG_REGION_MS
+    tf_key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+    meas_tf = peaks.get(tf_key, FALLBACK[tf_key])
     meas_bw = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
     line = {
         "metric": METRIC,
@@ -403,7 +409,8 @@ def run_ours(args, world, rank, local, dist):
         "frac_of_nominal_bf16": pf_tflops_1 / NOMINAL_BF16_TFLOPS,
         "roofline": {"bound": "tensor", "kernel": "attn::attn_fwd_kernel<128, false, false>",
                      "achieved": pf_tflops_1, "peak": meas_tf, "unit": "TFLOP/s", "frac": pf_tflops_1 / meas_tf,
-                     "peak_source": f"{peak_src} bf16 burst (cuBLAS)",
+                     "peak_source": f"{peak_src} bf16 {'sustained' if long_region else 'burst'} (cuBLAS; timed "
+                                    f"region {total_ms / 1e3:.2f} s)",
                      "traffic": ncu_traffic(P.name), "traffic_source": "ncu dram__bytes_read.sum + "
                      "dram__bytes_write.sum of one launch on this workload (null: not measured on this source)"},
         "decode": {
