@@ -49,7 +49,7 @@ PREFILL_SRC = "exact_io_aware_41_b200/csrc/attn_fwd.cu"
 DECODE_SRC = "exact_io_aware_41_b200/csrc/attn_decode.cu"
 PREFILL_SHA = "63b6180f1f6afe9c54d540d7fed48ed998708272751ad149f087cb68eb2d9625"  # sha256 of PREFILL_SRC when the prefill figures were taken
 BACKWARD_SRC = "exact_io_aware_41_b200/csrc/attn_bwd.cu"
-BACKWARD_SHA = "3adaec6fdcb10b13e4ac9fb4c0c81a7db88880515d94b87135bad0d662daae8f"
+BACKWARD_SHA = "7491f9ddae8c644559ef9b6c2c8b785dd6d0e2b6edefb74273e7b734d4d89e0d"
 NCU_TRAFFIC = {
     # attn_fwd_kernel<128>: 350.77 MB read + 52.83 MB written
     synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 403_600_640.0),
@@ -72,7 +72,7 @@ NCU_TRAFFIC = {
     # attn_fwd_kernel<128, 8-bit> on the long non-causal workload: 138.46 MB read + 42.28 MB written
     "fp8 " + synth.LONG_8K.name: (PREFILL_SRC, PREFILL_SHA, 180_734_720.0),
     # attn_bwd_kernel on the causal N2048 workload: 425.18 MB read + 215.12 MB written
-    "backward " + synth.CAUSAL_2K.name: (BACKWARD_SRC, BACKWARD_SHA, 658_183_936.0),
+    "backward " + synth.CAUSAL_2K.name: (BACKWARD_SRC, BACKWARD_SHA, 657_230_848.0),
     # decode_split_tc_kernel<128,4> (2123.81 MB read + 7.59 MB written) + decode_combine_kernel<128>
     # (4.29 MB read) on the full decode workload
     synth.DECODE.name: (DECODE_SRC, "eaf4990882bbcba5d723de8f5b505ab0c1520f88553cb35fa7ee6758aa501c3a", 2_135_693_824.0),

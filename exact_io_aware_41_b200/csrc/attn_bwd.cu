@@ -319,10 +319,11 @@ __global__ void __launch_bounds__(bwd::THREADS, 1)
     // ================================ dQ warps ================================
     // Per step, thread = query row q0 + row: once the dQ product is done, read it from TMEM (columns
     // 64..127 first, staged at once into the step's dO tile, read last by dV, done; then 0..63, after
-    // which the columns are released once dK is done too) and stage it as four 32 x 32 fp32 boxes
-    // (128-byte rows, swizzled like the tensor map): box c of this warp at c * 16 KB + wq * 4 KB, so
-    // boxes 0 and 1 land in the Q tile, which they may overwrite once dK (its last reader) is done. The TMA unit adds the boxes
-    // into the fp32 accumulator; once it has read them the buffer goes back to the producer.
+    // which the columns are released) and stage it as four 32 x 32 fp32 boxes (128-byte rows,
+    // swizzled like the tensor map): box c of this warp at c * 16 KB + wq * 4 KB, so boxes 0 and 1
+    // land in the Q tile, which they may overwrite once dK (its last reader) is done. The TMA unit
+    // adds the boxes into the fp32 accumulator; once it has read them the buffer goes back to the
+    // producer.
     regs_dec<DQ_REGS>();
     const int wq = warp & 3;
     const uint32_t lane_addr = tmem + (uint32_t(wq * 32) << 16);
