@@ -92,6 +92,15 @@ def ncu_traffic(name: str):
         return None
 
 
+def step_tensor_peak(peaks: dict, timed_ms: float):
+    """The bf16 tensor peak for a kernel timed inside the step loop: over a timed region of a second
+    or more the GPU settles at its power-capped clock, so the sustained GEMM figure; over a short one
+    (a few tens of steps) the burst figure. Returns (peak, long_region)."""
+    long_region = timed_ms >= LONG_REGION_MS
+    key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+    return peaks.get(key, FALLBACK[key]), long_region
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -378,12 +387,7 @@ def run_ours(args, world, rank, local, dist):
         dv, dsample, _ = cpu_decode(Dw, args.cpu_budget / 2)
         cpu["decode"] = {"value": dv, "unit": "GB/s", "sample": dsample}
 
-    # the headline kernel is timed inside the step loop: over a seconds-long timed region the GPU
-    # settles at its power-capped clock, so the denominator is the sustained GEMM figure; over a
-    # short one (a few tens of steps) it is the burst figure
-    long_region = total_ms >= LONG_REGION_MS
-    tf_key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
-    meas_tf = peaks.get(tf_key, FALLBACK[tf_key])
+    meas_tf, long_region = step_tensor_peak(peaks, total_ms)
     meas_bw = peaks.get("hbm_gbs", FALLBACK["hbm_gbs"])
     line = {
         "metric": METRIC,

@@ -76,3 +76,12 @@ def test_prefill_algorithmic_bytes():
 
 def test_max_over_ranks_single_process():
     assert bench.max_over_ranks([1.5, 2.0], None) == [1.5, 2.0]
+
+
+def test_step_peak_is_sustained_for_long_timed_regions():
+    measured = {"bf16_tflops": 1631.8, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6545.6}
+    assert bench.step_tensor_peak(measured, 27.0) == (1631.8, False)
+    assert bench.step_tensor_peak(measured, 2700.0) == (1400.0, True)
+    assert bench.step_tensor_peak(measured, bench.LONG_REGION_MS) == (1400.0, True)
+    # a peaks file without the sustained figure falls back to the recipe's one
+    assert bench.step_tensor_peak({"bf16_tflops": 1631.8}, 2700.0) == (bench.FALLBACK["bf16_tflops_sustained"], True)
