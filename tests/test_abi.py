@@ -125,3 +125,48 @@ def test_decode_sizes_the_combine_cannot_take_are_refused_before_any_launch(raw)
     # one split fewer passes the check and reaches the workspace check (too small here)
     assert lib.attn_decode_splitkv(p, p, p, p, cap - 64, p, p, 1, 1, 1, 32, 0.1, 64, p, 16, None) == \
         pkg.ATTN_ERR_WORKSPACE
+
+
+def test_backward_and_8bit_argument_errors_are_reported_before_any_launch(raw):
+    """The backward and 8-bit entry points refuse bad arguments on the host, before any CUDA call."""
+    import exact_io_aware_41_b200 as pkg
+
+    lib = pkg.lib_handle()
+    p = 1 << 20  # aligned, never dereferenced
+    big = 1 << 40
+
+    def bwd(*, q=p, lse=p, B=1, Hq=2, Hkv=2, Nq=16, Nkv=16, d=128, scale=0.125, causal=0, ws=p, ws_bytes=big):
+        return lib.attn_bwd(q, p, p, p, lse, p, p, p, p, B, Hq, Hkv, Nq, Nkv, d, scale, causal, ws, ws_bytes, None)
+
+    assert bwd(q=0) == pkg.ATTN_ERR_INVALID_ARG
+    assert bwd(q=p + 8) == pkg.ATTN_ERR_INVALID_ARG           # operands 16-byte aligned
+    assert bwd(lse=p + 2) == pkg.ATTN_ERR_INVALID_ARG         # lse 4-byte aligned
+    assert bwd(Hq=3) == pkg.ATTN_ERR_INVALID_ARG              # Hq a multiple of Hkv
+    assert bwd(Nkv=0) == pkg.ATTN_ERR_INVALID_ARG
+    assert bwd(scale=0.0) == pkg.ATTN_ERR_INVALID_ARG
+    assert bwd(causal=3) == pkg.ATTN_ERR_INVALID_ARG
+    assert bwd(d=64) == pkg.ATTN_ERR_UNSUPPORTED
+    assert bwd(ws=0) == pkg.ATTN_ERR_WORKSPACE
+    assert bwd(ws=p + 16) == pkg.ATTN_ERR_WORKSPACE           # workspace 256-byte aligned
+    assert bwd(ws_bytes=pkg.attn_bwd_workspace_bytes(1, 2, 16, 128) - 1) == pkg.ATTN_ERR_WORKSPACE
+    # 8-bit quantization and attention
+    assert lib.attn_fp8_quantize(0, None, p, p, 1, 16, 2, 128, 0, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fp8_quantize(p, None, p, p + 2, 1, 16, 2, 128, 0, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fp8_quantize(p, None, p, p, 1, 20, 2, 128, 1, None) == pkg.ATTN_ERR_INVALID_ARG  # N % 16
+    assert lib.attn_fp8_quantize(p, None, p, p, 1, 16, 2, 128, 2, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fp8_quantize(p, None, p, p, 1, 16, 2, 64, 0, None) == pkg.ATTN_ERR_UNSUPPORTED
+    f8 = [p, p, p, p, p, p, p, p]
+    assert lib.attn_fwd_fp8(*f8, 1, 2, 2, 16, 24, 128, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG  # Nkv % 16
+    assert lib.attn_fwd_fp8(*f8, 1, 3, 2, 16, 16, 128, 0.125, 0, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_fp8(*f8, 1, 2, 2, 16, 16, 128, float("inf"), 0, None) == pkg.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_fp8(*f8, 1, 2, 2, 16, 16, 64, 0.125, 0, None) == pkg.ATTN_ERR_UNSUPPORTED
+
+
+def test_backward_workspace_sizing():
+    import exact_io_aware_41_b200 as pkg
+
+    # fp32 dQ accumulator [B, Nq, Hq, d] rounded up to 256 bytes, then LSE' and D rows of whole
+    # 128-row tiles: B=2, Hq=3, Nq=130, d=128 -> 399360 + 2 * 2*3*256*4 = 411648
+    assert pkg.attn_bwd_workspace_bytes(2, 3, 130, 128) == 2 * 130 * 3 * 128 * 4 + 2 * (2 * 3 * 256 * 4)
+    assert pkg.attn_bwd_workspace_bytes(1, 1, 1, 128) == 512 + 2 * 128 * 4
+    assert pkg.attn_bwd_workspace_bytes(0, 1, 1, 128) == 0
