@@ -618,12 +618,14 @@ __global__ void __launch_bounds__(FwdCfg<D, F8, PAIR>::THREADS, 1)
           pos = base + 2 * n;
         }
         if (!ok) break;
-        // O may be read once every MMA writing it is done (one o_final phase per tile and unit), here
-        // after the unit's last PV. When tile 0 needs fewer K/V tiles (causal) its phase came right
-        // after its own last PV instead, so its epilogue runs during tile 1's last step. (Q was
-        // released after the unit's last QK, so the next unit's Q load overlaps the last PVs and the
-        // epilogues.)
-        if (C::NQT == 1 || un.n_tile0 == 0 || un.n_tile0 == n) commit(&o_final[0]);
+        // O may be read once every MMA writing it is done (one o_final phase per tile and unit with
+        // keys for that tile), here after the unit's last PV. When tile 0 needs fewer K/V tiles
+        // (causal) its phase came right after its own last PV instead, so its epilogue runs during
+        // tile 1's last step. A tile without keys gets no phase: its warpgroup takes no part in the
+        // unit, so phases committed for it could run two ahead of its waits, which a parity wait
+        // cannot tell apart. (Q was released after the unit's last QK, so the next unit's Q load
+        // overlaps the last PVs and the epilogues.)
+        if (C::NQT == 1 || un.n_tile0 == n) commit(&o_final[0]);
         if (C::NQT == 2) commit(&o_final[1]);
       }
       if (!ok) {
@@ -863,12 +865,8 @@ __global__ void __launch_bounds__(FwdCfg<D, F8, PAIR>::THREADS, 1)
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(args.o) +
                             ((size_t(un.b) * args.Nq + (valid ? q_row : 0)) * args.Hq + un.h) * D;
       if (un.n_tiles > 0 && my_tiles == 0) {
-        // this tile saw no key, but the unit had MMAs: keep the o_final phase count in step
-        if (!wait_warp(&o_final[qt], uint32_t(uc & 1))) {
-          ok = false;
-          break;
-        }
-        ++uc;
+        // this tile saw no key: O = 0 (no MMA wrote its accumulator, and no o_final phase was
+        // committed for it)
         if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow);
           for (int v4 = 0; v4 < D / 8; ++v4) dst[v4] = make_uint4(0, 0, 0, 0);

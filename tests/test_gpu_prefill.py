@@ -55,6 +55,13 @@ def test_edge_shapes_other_head_dims(lib, d):
     _run_small(lib, 3200 + d, 1, 2, 2, 200, 70, d, True)
 
 
+def test_many_units_whose_first_tile_has_no_key(lib):
+    # causal, Nq - Nkv = 400: per head, the 256-row block 0 sees no key, block 1's first 128 rows see
+    # none (its second tile does) and block 2 sees all; 4 x 32 heads give 384 units on at most 148
+    # CTAs, the light ones last, so CTAs take several keyless-first-tile units in a row
+    _run_small(lib, 4600, 4, 32, 8, 600, 200, 128, True)
+
+
 def test_gqa_group_of_eight_causal(lib):
     _run_small(lib, 4000, 1, 8, 1, 384, 384, 128, True)
 
