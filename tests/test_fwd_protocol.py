@@ -21,13 +21,17 @@ STAGES, SCHED = 4, 4
 ROLES = {"producer", "mma", "softmax0", "softmax1"}
 
 
-def forward_cta(sim, units, early_q_release=False, no_final_wait=False, phase_for_keyless_tile=False):
-    """units: (n, n0) per unit: K/V tiles of the unit and of its first query tile.
+def forward_cta(sim, units, early_q_release=False, no_final_wait=False, phase_for_keyless_tile=False,
+                sep_p=False, no_p_free_wait=False):
+    """units: (n, n0) per unit: K/V tiles of the unit and of its first query tile. sep_p: the d <= 64
+    variant, P in tensor-memory buffers of its own, the next S computed while the softmax works on
+    the current one (s_free: S read out; p_free: the PV reading the P buffer is done).
 
     The other arguments plant mistakes (for the tests that show the model catches them): Q released
     after the unit's first QK instead of its last; the second tile's O read out without waiting for
-    the unit's last product; and an o_final phase committed (and waited for) also for a first tile
-    without keys, whose warpgroup then takes no part in the unit."""
+    the unit's last product; an o_final phase committed (and waited for) also for a first tile
+    without keys, whose warpgroup then takes no part in the unit; and (sep_p) P written into its
+    buffer without waiting for the previous PV that reads it."""
     sim.bar("q_full")
     sim.bar("q_empty")
     for s in range(STAGES):
@@ -37,6 +41,8 @@ def forward_cta(sim, units, early_q_release=False, no_final_wait=False, phase_fo
         sim.bar(f"s_full{i}")
         sim.bar(f"p_full{i}")
         sim.bar(f"o_final{i}")
+        sim.bar(f"s_free{i}")
+        sim.bar(f"p_free{i}")
     for i in range(SCHED):
         sim.bar(f"sched_full{i}")
         sim.bar(f"sched_empty{i}", 3)  # the MMA issuer and the two softmax warpgroups
@@ -76,6 +82,9 @@ def forward_cta(sim, units, early_q_release=False, no_final_wait=False, phase_fo
         yield ("arrive", f"sched_empty{slot}")
 
     def mma():
+        if sep_p:
+            yield from mma_sep_p()
+            return
         qc, pos, pc = 0, 0, [0, 0]
         for k in range(end + 1):
             yield from consume_slot(k)
@@ -129,9 +138,67 @@ def forward_cta(sim, units, early_q_release=False, no_final_wait=False, phase_fo
                 yield ("commit", "o_final0")
             yield ("commit", "o_final1")
 
+    def mma_sep_p():
+        qc, pos, pc, qk_cnt = 0, 0, [0, 0], [0, 0]
+        for k in range(end + 1):
+            yield from consume_slot(k)
+            u = unit(k)
+            if u is None:
+                break
+            n, n0 = u
+            if n == 0:
+                continue
+            yield ("wait", "q_full", qc)
+            qc += 1
+            base = pos
+            nt = (n0, n)
+
+            def qk_into(qt, jj, stage_pos):
+                if qk_cnt[qt] > 0:
+                    yield ("wait", f"s_free{qt}", qk_cnt[qt] - 1)   # S read out by the softmax
+                yield ("mma", [("Q", f"Q {k}"), (f"KV{stage_pos % STAGES}", f"K{jj} u{k}")],
+                       [(f"S{qt}", f"S {qt} {jj} u{k}")])
+                yield ("commit", f"s_full{qt}")
+                if qt == 1 and jj == n - 1:
+                    yield ("commit", "q_empty")
+                qk_cnt[qt] += 1
+
+            yield ("wait", f"kv_full{base % STAGES}", base // STAGES)
+            for qt in range(2):
+                if nt[qt] > 0:
+                    yield from qk_into(qt, 0, base)
+            yield ("commit", f"kv_empty{base % STAGES}")
+            for j in range(n):
+                pv, pk = base + 2 * j + 1, base + 2 * j + 2
+                nxt = j + 1 < n
+                yield ("wait", f"kv_full{pv % STAGES}", pv // STAGES)
+                if nxt:
+                    yield ("wait", f"kv_full{pk % STAGES}", pk // STAGES)
+                for qt in range(2):
+                    if j + 1 < nt[qt]:
+                        yield from qk_into(qt, j + 1, pk)
+                for qt in range(2):
+                    if j >= nt[qt]:
+                        continue
+                    yield ("wait", f"p_full{qt}", pc[qt])
+                    pc[qt] += 1
+                    acc = [(f"O{qt}", f"O {qt} u{k}")] if j > 0 else []
+                    yield ("mma", [(f"P{qt}", f"P {qt} {j} u{k}"), (f"KV{pv % STAGES}", f"V{j} u{k}")] + acc,
+                           [(f"O{qt}", f"O {qt} u{k}")])
+                    yield ("commit", f"p_free{qt}")
+                    if qt == 0 and j == n0 - 1 and n0 < n:
+                        yield ("commit", "o_final0")
+                yield ("commit", f"kv_empty{pv % STAGES}")
+                if nxt:
+                    yield ("commit", f"kv_empty{pk % STAGES}")
+            pos = base + 2 * n
+            if n0 == n or (phase_for_keyless_tile and n0 == 0):
+                yield ("commit", "o_final0")
+            yield ("commit", "o_final1")
+
     def softmax(qt):
         rng = random.Random(sim.rng.random())
-        sc, uc = 0, 0
+        sc, uc, pt = 0, 0, 0
         for k in range(end + 1):
             yield from consume_slot(k)
             u = unit(k)
@@ -143,13 +210,23 @@ def forward_cta(sim, units, early_q_release=False, no_final_wait=False, phase_fo
                 yield ("wait", f"s_full{qt}", sc)
                 sc += 1
                 yield ("access", [(f"S{qt}", f"S {qt} {j} u{k}")], [], 1.0)
+                if sep_p:
+                    yield ("arrive", f"s_free{qt}")                           # the next QK may overwrite S
                 yield ("delay", 1.0)                                          # max
                 if j > 0 and rng.random() < 0.3:                              # O rescale in place
+                    if sep_p and pt > 0:
+                        yield ("wait", f"p_free{qt}", pt - 1)                 # the previous PV has landed
                     yield ("access", [(f"O{qt}", f"O {qt} u{k}")], [], 0.5)
                     yield ("access", [], [(f"O{qt}", f"O {qt} u{k}")], 0.5)
                 yield ("delay", 4.0)                                          # exponentials
-                yield ("access", [], [(f"S{qt}", f"P {qt} {j} u{k}")], 1.0)  # P over S
+                if sep_p:
+                    if pt > 0 and not no_p_free_wait:
+                        yield ("wait", f"p_free{qt}", pt - 1)                 # the P buffer is free again
+                    yield ("access", [], [(f"P{qt}", f"P {qt} {j} u{k}")], 1.0)
+                else:
+                    yield ("access", [], [(f"S{qt}", f"P {qt} {j} u{k}")], 1.0)  # P over S
                 yield ("arrive", f"p_full{qt}")
+                pt += 1
             if n == 0 or (my == 0 and not phase_for_keyless_tile):
                 continue                                                      # no key: zeros, no wait
             if not (no_final_wait and qt == 1):
@@ -235,3 +312,21 @@ def test_the_model_catches_a_phase_for_a_keyless_first_tile():
 def test_the_model_catches_a_read_out_before_the_last_product():
     """Planted mistake (in the model): the second tile's O read out without waiting for o_final."""
     assert _caught(60, no_final_wait=True) > 0
+
+
+@pytest.mark.parametrize("n_units", [1, 3, 9])
+def test_forward_protocol_with_separate_p_buffers(n_units):
+    for seed in range(80):
+        rng = random.Random(9000 + 100 * n_units + seed)
+        units = random_units(rng, n_units)
+        sim = Sim(seed)
+        forward_cta(sim, units, sep_p=True)
+        sim.go()
+        assert sim.finished == ROLES, f"units {units}, seed {seed}: left waiting {sorted(ROLES - sim.finished)}"
+        assert sim.pipe_done == sim.pipe_issued
+
+
+def test_the_model_catches_a_p_buffer_written_under_its_pv():
+    """Planted mistake (in the model, d <= 64 variant): P written into its buffer without waiting for
+    the previous PV, which may still be reading it."""
+    assert _caught(60, sep_p=True, no_p_free_wait=True) > 0
