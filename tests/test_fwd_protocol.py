@@ -330,3 +330,143 @@ def test_the_model_catches_a_p_buffer_written_under_its_pv():
     """Planted mistake (in the model, d <= 64 variant): P written into its buffer without waiting for
     the previous PV, which may still be reading it."""
     assert _caught(60, sep_p=True, no_p_free_wait=True) > 0
+
+
+PAIR_STAGES = 5
+PAIR_ROLES = {"producer0", "producer1", "mma", "softmax0", "softmax1"}
+
+
+def pair_cta(sim, units, rescale_without_o_done=False):
+    """The d = 256 variant on a CTA pair: one query tile of 128 rows per CTA (a 256-row unit), S
+    alternating between two slots (QK_0, QK_1, PV_0, QK_2, PV_1, ...), 2-SM products issued by the
+    leader that read and write both CTAs' halves, each CTA's producer loading its own halves with
+    the completion counted on the leader's barriers, commits reaching both CTAs. units: K/V tiles
+    per unit (the pair's units are a fixed list). rescale_without_o_done plants a mistake: O
+    rescaled without waiting for the previous PV."""
+    sim.bar("q_full", 2)
+    sim.bar("q_empty")
+    for st in range(PAIR_STAGES):
+        sim.bar(f"kv_full{st}", 2)
+        sim.bar(f"kv_empty{st}")
+    for i in range(2):
+        sim.bar(f"s_full{i}")
+        sim.bar(f"p_full{i}", 2)  # one arrival per CTA's softmax warpgroup
+    sim.bar("o_done")
+    sim.bar("o_final0")
+
+    def producer(r):
+        qc, pos = 0, 0
+        for k, n in enumerate(units):
+            if n == 0:
+                continue
+            if qc > 0:
+                yield ("wait", "q_empty", qc - 1)
+            yield ("async", [], [(f"Q_{r}", f"Q {k}")], 4.0, lambda: sim.arrive("q_full"))
+            qc += 1
+            for j in range(n):
+                for kv in ("K", "V"):
+                    st = pos % PAIR_STAGES
+                    yield ("wait", f"kv_empty{st}", pos // PAIR_STAGES - 1)
+                    yield ("async", [], [(f"KV{st}_{r}", f"{kv}{j} u{k}")], 3.0,
+                           (lambda st=st: sim.arrive(f"kv_full{st}")))
+                    pos += 1
+
+    def both(name, tag):
+        return [(f"{name}_0", tag), (f"{name}_1", tag)]
+
+    def mma():
+        qc, pos, t_run = 0, 0, 0
+        for k, n in enumerate(units):
+            if n == 0:
+                continue
+            yield ("wait", "q_full", qc)
+            qc += 1
+            base, t0 = pos, t_run
+            for j in range(min(2, n)):
+                kp = base + 2 * j
+                yield ("wait", f"kv_full{kp % PAIR_STAGES}", kp // PAIR_STAGES)
+                slot = (t0 + j) & 1
+                yield ("mma", both("Q", f"Q {k}") + both(f"KV{kp % PAIR_STAGES}", f"K{j} u{k}"),
+                       both(f"S{slot}", f"S {j} u{k}"))
+                yield ("commit", f"s_full{slot}")
+                if j == n - 1:
+                    yield ("commit", "q_empty")
+                yield ("commit", f"kv_empty{kp % PAIR_STAGES}")
+            for j in range(n):
+                t = t0 + j
+                slot = t & 1
+                vp = base + 2 * j + 1
+                yield ("wait", f"kv_full{vp % PAIR_STAGES}", vp // PAIR_STAGES)
+                yield ("wait", f"p_full{slot}", t >> 1)
+                acc = both("O", f"O u{k}") if j > 0 else []
+                yield ("mma", both(f"S{slot}", f"P {j} u{k}") + both(f"KV{vp % PAIR_STAGES}", f"V{j} u{k}") + acc,
+                       both("O", f"O u{k}"))
+                yield ("commit", "o_done")
+                yield ("commit", f"kv_empty{vp % PAIR_STAGES}")
+                if j + 2 < n:
+                    kp = base + 2 * (j + 2)
+                    yield ("wait", f"kv_full{kp % PAIR_STAGES}", kp // PAIR_STAGES)
+                    yield ("mma", both("Q", f"Q {k}") + both(f"KV{kp % PAIR_STAGES}", f"K{j + 2} u{k}"),
+                           both(f"S{slot}", f"S {j + 2} u{k}"))
+                    yield ("commit", f"s_full{slot}")
+                    if j + 3 == n:
+                        yield ("commit", "q_empty")
+                    yield ("commit", f"kv_empty{kp % PAIR_STAGES}")
+            t_run = t0 + n
+            pos = base + 2 * n
+            yield ("commit", "o_final0")
+
+    def softmax(r):
+        rng = random.Random(sim.rng.random())
+        t_run, uc = 0, 0
+        for k, n in enumerate(units):
+            for j in range(n):
+                slot = t_run & 1
+                yield ("wait", f"s_full{slot}", t_run >> 1)
+                t_run += 1
+                yield ("access", [(f"S{slot}_{r}", f"S {j} u{k}")], [], 1.0)
+                yield ("delay", 1.0)
+                if j > 0 and rng.random() < 0.3:
+                    if not rescale_without_o_done:
+                        yield ("wait", "o_done", t_run - 2)                   # the previous PV has landed
+                    yield ("access", [(f"O_{r}", f"O u{k}")], [], 0.5)
+                    yield ("access", [], [(f"O_{r}", f"O u{k}")], 0.5)
+                yield ("delay", 4.0)
+                yield ("access", [], [(f"S{slot}_{r}", f"P {j} u{k}")], 1.0)  # P over S
+                yield ("arrive", f"p_full{slot}")
+            if n == 0:
+                continue
+            yield ("wait", "o_final0", uc)
+            uc += 1
+            yield ("access", [(f"O_{r}", f"O u{k}")], [], 2.0)
+
+    for name, gen in (("producer0", producer(0)), ("producer1", producer(1)), ("mma", mma()),
+                      ("softmax0", softmax(0)), ("softmax1", softmax(1))):
+        sim.run(name, gen)
+
+
+@pytest.mark.parametrize("n_units", [1, 2, 5])
+def test_pair_protocol_has_no_hazard_and_finishes(n_units):
+    for seed in range(80):
+        rng = random.Random(11000 + 100 * n_units + seed)
+        units = [rng.choice((0, 1, 2, 3, 5, 8)) for _ in range(n_units)]
+        sim = Sim(seed)
+        pair_cta(sim, units)
+        sim.go()
+        assert sim.finished == PAIR_ROLES, f"units {units}, seed {seed}: left waiting {sorted(PAIR_ROLES - sim.finished)}"
+        assert sim.pipe_done == sim.pipe_issued
+
+
+def test_the_model_catches_a_pair_rescale_without_o_done():
+    caught = 0
+    for seed in range(60):
+        sim = Sim(seed)
+        pair_cta(sim, [4, 6, 3], rescale_without_o_done=True)
+        try:
+            sim.go()
+        except Hazard:
+            caught += 1
+            continue
+        if sim.finished != PAIR_ROLES:
+            caught += 1
+    assert caught > 0
