@@ -159,6 +159,10 @@ __device__ __forceinline__ void warp_publish_tmem_stores(uint64_t* bar, int lane
 constexpr int kSchedSlots = 256;
 __device__ unsigned int g_sched_next[kSchedSlots];
 __device__ unsigned int g_sched_done[kSchedSlots];
+// The slots are shared by every variant of the kernel (head dims, 8-bit), so one launch counter
+// serves them all: two launches in flight on different streams never get the same slot, whatever
+// variants they are (up to kSchedSlots launches in flight).
+static std::atomic<unsigned> g_fwd_launch_count{0};
 
 // Units in issue order: heads grouped so a group's K/V fit comfortably in L2 (group size chosen on
 // the host) and, inside a group, heaviest first (every head's last query block, then the one
@@ -1045,8 +1049,7 @@ static attn_status_t launch_fwd(const void* q, const void* k, const void* v, voi
   }
   // persistent grid: one CTA per SM (each holds all 512 TMEM columns), walking the units in order
   const unsigned grid = unsigned(units < sms ? units : sms);
-  static std::atomic<unsigned> launch_count{0};
-  a.sched_slot = int(launch_count.fetch_add(1) % kSchedSlots);
+  a.sched_slot = int(g_fwd_launch_count.fetch_add(1) % kSchedSlots);
   kernel<<<dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, a);
   return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : (cudaGetLastError(), ATTN_ERR_CUDA);
 }
